@@ -1,0 +1,134 @@
+// lbq_common.cuh -- device helpers shared by the liblbq kernels (sm_100a).
+#pragma once
+#include <cstdint>
+#include <type_traits>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include "../../include/lbq.h"
+
+namespace lbq {
+
+// Device error word bits (read back by lbq_last_device_error).
+constexpr unsigned kErrNonFinite = 1u;
+constexpr unsigned kErrTimeout = 2u;
+
+// Address of this device's error word (set up once per device by the ABI layer).
+unsigned* device_error_word();
+int sm_count();
+
+// ---------------------------------------------------------------- loads
+// Streaming 128-bit load through the non-coherent path, not kept in L1.
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+// Read-only loads that may be cached in L1 (activations, scales).
+__device__ __forceinline__ uint32_t ldg_u32(const void* p) {
+    uint32_t r;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(r) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint2 ldg_u64(const void* p) {
+    uint2 r;
+    asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint4 ldg_u128(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint16_t ldg_u16(const void* p) {
+    unsigned short r;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));
+    return r;
+}
+
+// ---------------------------------------------------------------- bit ops
+// d = (a & b) | c   (one LOP3)
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+template <int S>
+__device__ __forceinline__ uint32_t shift_right_signed(uint32_t v) {
+    if constexpr (S > 0) return v >> S;
+    else if constexpr (S < 0) return v << (-S);
+    else return v;
+}
+
+// ---------------------------------------------------------------- half2 arithmetic on raw bits
+__device__ __forceinline__ uint32_t hsub2_f16(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t hsub2_bf16(uint32_t a, uint32_t b) {
+    // bf16x2 subtraction as a*1 - b (fma.rn.bf16x2 is native on sm_90+)
+    uint32_t d;
+    const uint32_t one = 0x3F803F80u;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(one), "r"(b ^ 0x80008000u));
+    return d;
+}
+
+// ---------------------------------------------------------------- legacy tensor-core MMA
+// D = A(16x16, row) * B(16x8, col) + C, fp16 or bf16 inputs, fp32 accumulators.
+template <bool BF16>
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    if constexpr (BF16) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    } else {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+}
+
+// D = A(16x32 u8, row) * B(32x8 s8, col) + C, int32 accumulators.
+__device__ __forceinline__ void mma_16832_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------- misc
+// Compile-time loop: f(std::integral_constant<int, I>) for I in [BEGIN, END).
+template <int BEGIN, int END, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+    if constexpr (BEGIN < END) {
+        f(std::integral_constant<int, BEGIN>{});
+        static_for<BEGIN + 1, END>(f);
+    }
+}
+
+__host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+template <bool BF16>
+__device__ __forceinline__ float to_f32(uint16_t v) {
+    if constexpr (BF16) return __uint_as_float(uint32_t(v) << 16);
+    else return __half2float(__ushort_as_half(v));
+}
+template <bool BF16>
+__device__ __forceinline__ uint16_t from_f32(float v) {
+    if constexpr (BF16) return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    else return __half_as_ushort(__float2half_rn(v));
+}
+
+inline lbq_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? LBQ_OK : LBQ_ERR_CUDA;
+}
+
+}  // namespace lbq

@@ -1,0 +1,79 @@
+// lbq_internal.h -- host-side launchers and layout geometry shared inside liblbq.
+#pragma once
+#include <algorithm>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include "../../include/lbq.h"
+
+namespace lbq {
+
+unsigned* device_error_word();
+int sm_count();
+
+// Geometry of the fragment-interleaved group-code layout (LBQ_LAYOUT_KERNEL).
+// A b-bit code is a low plane of W0 bits and a high plane of W1 = b - W0 bits.
+// Blocks of 512 bytes hold 16 rows x 256/w codes of one plane; a superblock of
+// SB = 256 / min(W0, W1) codes along k holds NB0 = SB*W0/256 low blocks then
+// NB1 = SB*W1/256 high blocks (SB_BYTES = 2*SB*b).
+template <int B>
+struct GroupGeom {
+    static constexpr int W0 = (B == 2 || B == 3) ? 2 : 4;
+    static constexpr int W1 = B - W0;
+    static constexpr int WMIN = (W1 > 0 && W1 < W0) ? W1 : W0;
+    static constexpr int SB = 256 / WMIN;
+    static constexpr int NB0 = SB * W0 / 256;
+    static constexpr int NB1 = SB * W1 / 256;
+    static constexpr int NBLK = NB0 + NB1;
+    static constexpr int SB_BYTES = 2 * SB * B;
+    static_assert(NBLK * 512 == SB_BYTES, "layout geometry");
+};
+
+inline int64_t group_superblock(int bits) {
+    switch (bits) {
+        case 2: return GroupGeom<2>::SB;
+        case 3: return GroupGeom<3>::SB;
+        case 4: return GroupGeom<4>::SB;
+        case 5: return GroupGeom<5>::SB;
+        case 6: return GroupGeom<6>::SB;
+        default: return 0;
+    }
+}
+
+inline int64_t sign_cols_pad(int64_t cols) { return (cols + 255) / 256 * 256; }
+
+// Every workspace starts with a fixed header of ticket counters (one per 16-row
+// tile, at most kMaxTiles).  It must be zero before the first call; every call
+// leaves it zero.  The bytes after it are scratch, always written before read.
+constexpr int64_t kMaxTiles = 16384;
+constexpr size_t kCounterBytes = (size_t)kMaxTiles * 4;
+
+lbq_status launch_quantize_rtn(const void* W, bool bf16, int64_t n, int64_t k, int bits, int group,
+                               uint8_t* codes, void* scales, void* zeros, cudaStream_t st);
+lbq_status launch_pack(const uint8_t* codes, int64_t n, int64_t k, int bits, lbq_layout layout, void* packed,
+                       cudaStream_t st);
+lbq_status launch_unpack(const void* packed, int64_t n, int64_t k, int bits, lbq_layout layout, uint8_t* codes,
+                         cudaStream_t st);
+lbq_status launch_pack_signs(const int8_t* pm1, int64_t rows, int64_t cols, lbq_layout layout, void* out,
+                             cudaStream_t st);
+lbq_status launch_repack_signs(const uint32_t* canon, int64_t rows, int64_t cols, void* out, cudaStream_t st);
+
+// Group GEMV (M <= 16).  ws layout and size: gemv_group_ws_bytes.
+size_t gemv_group_ws_bytes(int64_t M, int64_t n, int64_t k, int bits, lbq_layout layout);
+lbq_status launch_gemv_group(const void* x, bool bf16, int64_t M, const void* packed, const void* scales,
+                             const void* zeros, int64_t n, int64_t k, int bits, int group, lbq_layout layout,
+                             void* y, void* ws, size_t ws_bytes, cudaStream_t st);
+
+// Batched group GEMM on tcgen05 (M >= 64, kernel layout).
+size_t gemm_group_tc_ws_bytes(int64_t M, int64_t n, int64_t k);
+bool gemm_group_tc_supported(int64_t M, int64_t n, int64_t k, int bits, int group);
+lbq_status launch_gemm_group_tc(const void* x, bool bf16, int64_t M, const void* packed, const void* scales,
+                                const void* zeros, int64_t n, int64_t k, int bits, int group, void* y, void* ws,
+                                size_t ws_bytes, cudaStream_t st);
+
+// Binary low-rank GEMV (M <= 16).
+size_t gemv_binlr_ws_bytes(int64_t M, int64_t d_out, int64_t d_in, int64_t r, lbq_layout layout);
+lbq_status launch_gemv_binlr(const void* x, bool bf16, int64_t M, const void* U, const void* Vt, const void* s1,
+                             const void* s2, int64_t d_out, int64_t d_in, int64_t r, lbq_layout layout, void* y,
+                             void* ws, size_t ws_bytes, cudaStream_t st);
+
+}  // namespace lbq
