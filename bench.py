@@ -475,6 +475,37 @@ def run_gpu(args, dev):
         dist.destroy_process_group()
 
 
+def run_breakdown(args, dev):
+    """Per-linear device time of the block workload (stderr; analysis aid, not the bench line)."""
+    wk = WORKLOADS[args.workload](dev)
+    stream = torch.cuda.Stream(device=dev)
+    reps = 20
+    with torch.cuda.stream(stream):
+        for p, l in enumerate(wk.linears):
+            graphs = []
+            for c in range(wk.copies):
+                packed, s, z, _ = wk.sets[c][p] if args.workload == "block" else (None, None, None, None)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for _ in range(reps):
+                        wk.lbq.lbq_gemv_group(wk.x[p], packed, s, z, l.d_out, l.d_in, wk.bits, wk.group,
+                                              wk.lbq.LAYOUT_KERNEL, y=wk.y[p], ws=wk.ws)
+                graphs.append(g)
+            for c in range(wk.copies):
+                graphs[c].replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(8):
+                graphs[i % wk.copies].replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / (8 * reps)
+            byts = wl.gemv_algorithmic_bytes(l.d_out, l.d_in, wk.bits, wk.group, 1)
+            print(f"{l.name:10s} {l.d_out:6d}x{l.d_in:<6d} {us:8.2f} us  {byts / us / 1e3:8.1f} GB/s",
+                  file=sys.stderr, flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -483,13 +514,16 @@ def main():
     ap.add_argument("--impl", choices=["lbq", "reference"], default="lbq")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="block")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--breakdown", action="store_true", help="print per-linear device times to stderr and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     _, _, local = _rank_info()
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     if dev.type == "cuda":
         torch.cuda.set_device(dev)
-    if args.impl == "reference":
+    if args.breakdown:
+        run_breakdown(args, dev)
+    elif args.impl == "reference":
         run_reference(args, dev)
     else:
         if dev.type != "cuda":

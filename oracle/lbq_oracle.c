@@ -36,8 +36,9 @@
  *      stream bit j*b+t); sign packing: element c at bit c%32 of word
  *      c/32, bit 1 meaning +1;
  *  R8  the fragment-interleaved kernel layout is a permutation of the same
- *      bits; its index map is written out in orc_kernel_pos() below from the
- *      specification in DESIGN.md ("Kernel layout"), independently of the
+ *      bits (tiles of 16 rows x 256 columns in integer tensor-core fragment
+ *      order); its index map is written out in orc_kernel_pos() below from
+ *      the specification in DESIGN.md ("Kernel layout"), independently of the
  *      CUDA packer.
  *
  * Parity pins for every function live in tests/test_oracle_*.py; there is
@@ -231,21 +232,18 @@ int orc_unpack_canonical(const uint8_t* in, int64_t n, int64_t k, int bits, uint
 /*    of width w1 = b - w0: b=2 -> (2), b=3 -> (2,1), b=4 -> (4),              */
 /*    b=5 -> (4,1), b=6 -> (4,2).  Low plane value = q mod 2^w0, high plane   */
 /*    value = q >> w0.                                                        */
-/*  * rows are cut into tiles of 16; k into superblocks of SB = 256/min(w)    */
-/*    codes.  Superblock (T, S) occupies 2*SB*b bytes at byte offset          */
-/*    (T*(k/SB) + S) * 2*SB*b.  Inside it come the low-plane blocks, then     */
-/*    the high-plane blocks, each 512 bytes; a plane of width w has SB*w/256  */
-/*    blocks, block beta covering codes [S*SB + beta*256/w, +256/w).          */
-/*  * a block of width w spans 256/w codes of k, i.e. P = 16/w "slices" of  */
-/*    16 consecutive k.  Lane L = 0..31 (g = L/4, c = L%4) owns bytes         */
-/*    [16L, 16L+16) = little-endian words W0..W3.  W0 holds row g and W1 row  */
-/*    g+8 of slices [0, P/2); W2 holds row g and W3 row g+8 of slices          */
-/*    [P/2, P).  Half h of a word (bits 16h..16h+15) holds P codes of width   */
-/*    w; the one at position pi (bits 16h + w*pi .. ) is the code of          */
-/*    k = k_block + 16*(sigma0 + pi/2) + 2c + 8*(pi%2) + h, sigma0 being the  */
-/*    word's first slice.  (These are the m16n8k16 A-fragment slots 2c,      */
-/*    2c+1, 2c+8, 2c+9 of lane L, paired the way a 16-bit-half unpack yields  */
-/*    them.)                                                                  */
+/*  * rows are cut into tiles of 16 and k into superblocks of 256.  Tile T,   */
+/*    superblock S occupies 512*b bytes at byte offset (T*(k/256) + S)*512*b: */
+/*    first the low plane (512*w0 bytes), then the high plane (512*w1).       */
+/*  * element (row r = 16T + g + 8u, column k = 256S + 32*kappa + 8c + nu),   */
+/*    g in 0..7, u in 0..1, kappa in 0..7, c in 0..3, nu in 0..7, belongs to  */
+/*    lane L = 4g + c and octet eta = 2*kappa + u of that lane; nu = 2j + e.  */
+/*  * in a plane of width w a 32-bit word holds O = 4/w octets: octet        */
+/*    eta sits in word omega = eta / O as slot o = eta % O, and its code     */
+/*    nu = 2j + e occupies bits 8j + 2w*o + w*e .. +w-1.  Word omega of lane  */
+/*    L is at byte (omega/4)*512 + 16L + 4*(omega%4) of the plane.            */
+/*    (Masking a word with 0x0F0F0F0F-style byte masks after a shift yields   */
+/*    the m16n8k32 u8 A-fragment registers of lane L directly.)               */
 /* ------------------------------------------------------------------------- */
 
 static void plane_widths(int bits, int* w0, int* w1)
@@ -261,10 +259,8 @@ static void plane_widths(int bits, int* w0, int* w1)
 
 static int superblock_k(int bits)
 {
-    int w0, w1;
-    plane_widths(bits, &w0, &w1);
-    int wmin = (w1 > 0 && w1 < w0) ? w1 : w0;
-    return 256 / wmin;
+    (void)bits;
+    return 256;
 }
 
 /* For element (row i, column kk) and plane index pl (0 low, 1 high), return
@@ -274,27 +270,19 @@ static int64_t orc_kernel_pos(int64_t i, int64_t kk, int64_t k, int bits, int pl
     int w0, w1;
     plane_widths(bits, &w0, &w1);
     const int w = pl == 0 ? w0 : w1;
-    const int64_t SB = superblock_k(bits);
     const int64_t T = i / 16, r = i % 16;
-    const int64_t S = kk / SB, ks = kk % SB;       /* position inside superblock */
-    int64_t off = (T * (k / SB) + S) * (2 * SB * bits);    /* bytes */
-    if (pl == 1) off += (SB * w0 / 256) * 512;     /* skip low-plane blocks */
-    const int64_t span = 256 / w;                  /* codes per block */
-    const int64_t beta = ks / span, kb = ks % span;
-    off += beta * 512;
-    const int P = 16 / w;                          /* slices per block */
-    const int64_t sigma = kb / 16, s = kb % 16;    /* slice, slot */
-    /* slot s = 2c + 8*(pi%2) + h */
-    const int h = (int)(s & 1);
-    const int c = (int)((s % 8) / 2);
-    const int pi_odd = (int)(s / 8);
-    const int second = sigma >= P / 2;              /* W2/W3 vs W0/W1 */
-    const int64_t sigma_in_word = second ? sigma - P / 2 : sigma;
-    const int pi = (int)(2 * sigma_in_word + pi_odd);
-    const int g = (int)(r % 8), upper = (int)(r / 8);
+    const int g = (int)(r % 8), u = (int)(r / 8);
+    const int64_t S = kk / 256, ks = kk % 256;
+    const int kappa = (int)(ks / 32), c = (int)((ks % 32) / 8), nu = (int)(ks % 8);
+    const int j = nu / 2, e = nu % 2;
     const int lane = 4 * g + c;
-    const int word = 2 * second + upper;
-    return (off + 16 * lane + 4 * word) * 8 + 16 * h + w * pi;
+    const int eta = 2 * kappa + u;
+    const int O = 4 / w;
+    const int omega = eta / O, o = eta % O;
+    int64_t byte = (T * (k / 256) + S) * 512 * bits;
+    if (pl == 1) byte += 512 * w0;
+    byte += (omega / 4) * 512 + 16 * lane + 4 * (omega % 4);
+    return byte * 8 + 8 * j + 2 * w * o + w * e;
 }
 
 int orc_pack_kernel(const uint8_t* codes, int64_t n, int64_t k, int bits, uint8_t* out)

@@ -173,10 +173,12 @@ size_t lbq_workspace_bytes(lbq_op op, int64_t M, int64_t n, int64_t k, int64_t r
     if (M <= 0) return 0;
     switch (op) {
         case LBQ_OP_GEMV_GROUP: {
-            size_t best = 0;
+            size_t best = kCounterBytes;
             for (int b = 2; b <= 6; b++)
-                if (k % group_superblock(b) == 0 && n % 16 == 0)
-                    best = std::max(best, gemv_group_ws_bytes(std::min<int64_t>(M, 16), n, k, b, LBQ_LAYOUT_KERNEL));
+                for (int g = 32; g <= 128; g *= 2)
+                    if (k % group_superblock(b) == 0 && k % g == 0 && n % 16 == 0)
+                        best = std::max(best, gemv_group_ws_bytes(std::min<int64_t>(M, 16), n, k, b, g,
+                                                                  LBQ_LAYOUT_KERNEL));
             return best;
         }
         case LBQ_OP_GEMM_GROUP: {

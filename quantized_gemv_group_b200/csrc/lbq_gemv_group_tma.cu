@@ -1,0 +1,469 @@
+// lbq_gemv_group_tma.cu -- dequant-fused group GEMV on integer tensor cores (sm_100a), M = 1..16.
+//
+//   y[m, i] = sum_k x[m, k] * s[i, k/g] * (q[i, k] - z[i, k/g])
+//
+// Decode time per token is the bytes read over the read bandwidth ("AirLLM corre un
+// modelo 70B en una GPU de 4GB...", section "Por qué es lento"): the kernel must keep
+// HBM streaming while spending as few instructions per weight as possible.
+//
+//  * A producer warp streams each 256-wide k chunk of a 128-row block into a
+//    shared-memory ring with the Tensor Memory Accelerator: the eight 16-row tiles'
+//    packed codes (1-D bulk copies, evict-first in L2) on one transaction-count
+//    mbarrier, the activation rows (1-D bulk copies) and 128 x 8 tiles of the fp16
+//    scales and zeros (2-D tensor copies) on a second one, so that the activation
+//    prep of a stage starts while its weights are still in flight.
+//  * Launched as a programmatic dependent of the previous kernel in the stream, the
+//    producer issues the first stages' weight and scale copies before waiting for
+//    that kernel (griddepcontrol.wait); only the activation copies, the prep and the
+//    stores depend on it.  Packed weights, scales and zeros must therefore not be
+//    written by a kernel that signals programmatic completion early.
+//  * Two prep warps turn each activation chunk into 16-bit fixed point with one
+//    power-of-two scale 2^E per token and chunk (|v| <= 32639), split into int8
+//    planes hi, lo (v = 256 hi + lo) laid out for the B fragment, plus the per-group
+//    sums of v.
+//  * Eight consumer warps (one 16-row tile each) mask the packed words into u8 A
+//    fragments (one LOP per four codes) and run mma.m16n8k32 u8 x s8 -> s32, hi and
+//    lo planes side by side in the N dimension.  Per group the exact integer
+//    sum (q - z) v = S - z * sum(v) is scaled by s * 2^E into an fp32 accumulator.
+//  * CTAs split the (row block, k chunk) units evenly ("stream-K"); a row block split
+//    between CTAs is finished by the last CTA to arrive (tile_epilogue).
+//  * Every wait is bounded; on expiry the kernel records kErrTimeout, stops issuing,
+//    waits (bounded) for its own copies in flight and returns.
+// Group codes: "TurboQuant: cuantizar modelos grandes para que quepan en local",
+// section "Compresión por bloques"; RTN codes: "Métodos de cuantización de LLM para
+// ejecutar un modelo de 70B en una sola GPU", section "RTN (Round-To-Nearest)".
+#include <cuda.h>
+#include "lbq_common.cuh"
+#include "lbq_internal.h"
+#include "lbq_group_frag.cuh"
+
+namespace lbq {
+
+constexpr int kConsumers = 8;
+constexpr int kPrepWarps = 2;
+constexpr int kProducerWarp = kConsumers;
+constexpr int kGemvThreads = (kConsumers + 1 + kPrepWarps) * 32;
+constexpr int kChunk = 256;                            // k per pipeline stage
+constexpr int kPlanePitch = kChunk + 16;                // bytes per int8 plane row in smem (bank pad)
+constexpr int kScaleBox = 8;                            // groups per scale-tile row (a chunk never spans more)
+constexpr int kScaleTile = 128 * kScaleBox * 2;         // bytes of one 128 x 8 fp16 tile
+constexpr int kBarBytes = 512;                          // mbarriers + abort flag
+constexpr int kGemvSmemBudget = 110 * 1024;             // two CTAs per SM
+constexpr int kPlaneMaxAbs = 32639;                     // |v| bound so that (v + 128) >> 8 fits in int8
+
+struct StageLayout {
+    int w, xraw, planes, xsum, expo, sc, zr, bytes;
+    __host__ __device__ StageLayout(int B, int M) {
+        w = 0;
+        xraw = 128 * kChunk * B / 8;
+        planes = xraw + up(M * 2 * kChunk, 16);
+        xsum = planes + up(2 * M * kPlanePitch, 16);
+        expo = xsum + up(M * 8 * 4, 16);
+        sc = up(expo + up(M * 4, 16), 128);
+        zr = sc + kScaleTile;
+        bytes = zr + kScaleTile;
+    }
+    __host__ __device__ static int up(int v, int a) { return (v + a - 1) / a * a; }
+};
+
+// Smallest E with maxabs * 2^-E <= kPlaneMaxAbs (E = 0 for an all-zero chunk).
+__device__ __forceinline__ int fixed_point_exponent(float maxabs) {
+    if (!(maxabs > 0.0f)) return 0;
+    const int e0 = ilogbf(maxabs) - 14;
+    return e0 + (ldexpf(maxabs, -e0) > (float)kPlaneMaxAbs ? 1 : 0);
+}
+
+template <int B, int GROUP, int NB, bool BF16>
+__global__ void __launch_bounds__(kGemvThreads, 2)
+k_gemv_group_tc(const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_z,
+                const uint16_t* __restrict__ x, int M, const uint8_t* __restrict__ packed, int64_t n, int64_t k,
+                uint16_t* __restrict__ y, float* __restrict__ partials, unsigned* __restrict__ counters, int maxc,
+                int nstage, unsigned* err) {
+    using G = GroupGeom<B>;
+    using F = IFrag<B>;
+    constexpr int TILE_BYTES = G::SB_BYTES;            // one tile's codes per stage (512 * B)
+    constexpr int KPG = GROUP / 32;                    // k-steps per group
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);     // full[nstage] empty[nstage] xready[nstage]
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBarBytes - 4);
+    const StageLayout L(B, M);
+    uint8_t* stage0 = smem + kBarBytes;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t KCH = k / kChunk;
+    const int64_t n_tiles = n / 16;
+    const int64_t n_rb = ceil_div(n_tiles, kConsumers);
+    const int64_t S_total = n_rb * KCH;
+    const int64_t NC = gridDim.x;
+    const int64_t u_begin = (int64_t)blockIdx.x * S_total / NC;
+    const int64_t u_end = ((int64_t)blockIdx.x + 1) * S_total / NC;
+
+    // barriers: wfull[s] (weights), afull[s] (activations + scales), empty[s], xready[s]
+    auto wfull = [&](int s) { return smem_u32(&bars[s]); };
+    auto afull = [&](int s) { return smem_u32(&bars[nstage + s]); };
+    auto empty = [&](int s) { return smem_u32(&bars[2 * nstage + s]); };
+    auto xready = [&](int s) { return smem_u32(&bars[3 * nstage + s]); };
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nstage; s++) {
+            mbar_init(wfull(s), 1);
+            mbar_init(afull(s), 1);
+            mbar_init(empty(s), kConsumers);
+            mbar_init(xready(s), kPrepWarps);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    griddep_launch_dependents();
+
+    // ------------------------------------------------------------ producer warp
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_first();
+            // Issues the copies of unit u into stage s; the activation rows only when with_x.
+            auto issue = [&](int64_t u, int s, bool static_part, bool with_x) {
+                const int64_t rb = u / KCH, kc = u % KCH;
+                uint8_t* st = stage0 + (size_t)s * L.bytes;
+                if (static_part) {
+                    const int64_t tiles_left = n_tiles - rb * kConsumers;
+                    const int tiles = (int)(tiles_left < kConsumers ? tiles_left : kConsumers);
+                    mbar_arrive_expect_tx(wfull(s), (uint32_t)(tiles * TILE_BYTES));
+                    for (int t = 0; t < tiles; t++)
+                        tma_load_1d_hint(smem_u32(st + t * TILE_BYTES),
+                                         packed + ((rb * kConsumers + t) * KCH + kc) * (int64_t)TILE_BYTES,
+                                         TILE_BYTES, wfull(s), pol);
+                    mbar_arrive_expect_tx(afull(s), (uint32_t)(M * 2 * kChunk + 2 * kScaleTile));
+                    const int j0 = (int)((kc * kChunk) / GROUP) & ~7;
+                    tma_load_2d(smem_u32(st + L.sc), &tm_s, j0, (int)(rb * 128), afull(s));
+                    tma_load_2d(smem_u32(st + L.zr), &tm_z, j0, (int)(rb * 128), afull(s));
+                }
+                if (with_x)
+                    for (int m = 0; m < M; m++)
+                        tma_load_1d(smem_u32(st + L.xraw + m * 2 * kChunk), x + (int64_t)m * k + kc * kChunk,
+                                    2 * kChunk, afull(s));
+            };
+            // prologue: weights and scales of the first stages do not depend on the previous kernel
+            const int64_t pro = min((int64_t)nstage, u_end - u_begin);
+            for (int64_t j = 0; j < pro; j++) issue(u_begin + j, (int)j, true, false);
+            griddep_wait();
+            for (int64_t j = 0; j < pro; j++) issue(u_begin + j, (int)j, false, true);
+            int64_t it = pro;
+            for (int64_t u = u_begin + pro; u < u_end; u++, it++) {
+                const int s = (int)(it % nstage);
+                const uint32_t ph = (uint32_t)((it / nstage) & 1);
+                if (!mbar_wait_bounded(empty(s), ph ^ 1u, err)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                issue(u, s, true, true);
+            }
+            for (int64_t j = (it > nstage ? it - nstage : 0); j < it; j++) {
+                mbar_wait_bounded(wfull((int)(j % nstage)), (uint32_t)((j / nstage) & 1), err);
+                mbar_wait_bounded(afull((int)(j % nstage)), (uint32_t)((j / nstage) & 1), err);
+            }
+        } else {
+            griddep_wait();
+        }
+        return;
+    }
+
+    // ------------------------------------------------------------ activation prep warps
+    if (warp > kProducerWarp) {
+        const int pw = warp - kProducerWarp - 1;
+        int64_t it = 0;
+        for (int64_t u = u_begin; u < u_end; u++, it++) {
+            const int s = (int)(it % nstage);
+            const uint32_t ph = (uint32_t)((it / nstage) & 1);
+            if (*abort_flag || !mbar_wait_bounded(afull(s), ph, err)) {
+                *abort_flag = 1;
+                return;
+            }
+            uint8_t* st = stage0 + (size_t)s * L.bytes;
+            for (int m = pw; m < M; m += kPrepWarps) {
+                const uint4 raw = *reinterpret_cast<const uint4*>(st + L.xraw + m * 2 * kChunk + 16 * lane);
+                const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+                float v[8];
+                float mx = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 8; e++) {
+                    v[e] = to_f32<BF16>((uint16_t)(rw[e / 2] >> (16 * (e & 1))));
+                    mx = fmaxf(mx, fabsf(v[e]));
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                const int E = fixed_point_exponent(mx);
+                uint32_t hev = 0, hod = 0, lev = 0, lod = 0;
+                int sum = 0;
+#pragma unroll
+                for (int e = 0; e < 8; e++) {
+                    const int q = __float2int_rn(ldexpf(v[e], -E));
+                    const int h = (q + 128) >> 8;
+                    const int l = q - 256 * h;
+                    sum += q;
+                    const int sh = 8 * (e >> 1);
+                    if (e & 1) {
+                        hod |= (uint32_t)(h & 0xFF) << sh;
+                        lod |= (uint32_t)(l & 0xFF) << sh;
+                    } else {
+                        hev |= (uint32_t)(h & 0xFF) << sh;
+                        lev |= (uint32_t)(l & 0xFF) << sh;
+                    }
+                }
+                *reinterpret_cast<uint2*>(st + L.planes + (2 * m) * kPlanePitch + 8 * lane) = make_uint2(hev, hod);
+                *reinterpret_cast<uint2*>(st + L.planes + (2 * m + 1) * kPlanePitch + 8 * lane) = make_uint2(lev, lod);
+                constexpr int LPG = GROUP / 8;                 // lanes per group
+#pragma unroll
+                for (int o = 1; o < LPG; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                if (lane % LPG == 0) reinterpret_cast<int*>(st + L.xsum)[m * 8 + lane / LPG] = sum;
+                if (lane == 0) reinterpret_cast<int*>(st + L.expo)[m] = E;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xready(s));
+        }
+        return;
+    }
+
+    // ------------------------------------------------------------ consumer warps
+    const int g = lane >> 2, c = lane & 3;
+    const int rl = warp * 16 + g;                        // row inside the 128-row block
+    int64_t it = 0;
+    for (int64_t u0 = u_begin; u0 < u_end;) {
+        const int64_t rb = u0 / KCH;
+        const int64_t kc0 = u0 % KCH;
+        const int64_t kc1 = min(KCH, kc0 + (u_end - u0));
+        u0 += kc1 - kc0;
+        const int64_t tile = rb * kConsumers + warp;
+        const bool active = tile < n_tiles;
+
+        float acc[NB][2];
+#pragma unroll
+        for (int nb = 0; nb < NB; nb++) acc[nb][0] = acc[nb][1] = 0.0f;
+
+        for (int64_t kc = kc0; kc < kc1; kc++, it++) {
+            const int s = (int)(it % nstage);
+            const uint32_t ph = (uint32_t)((it / nstage) & 1);
+            if (!mbar_wait_bounded(wfull(s), ph, err) || !mbar_wait_bounded(xready(s), ph, err)) {
+                *abort_flag = 1;
+                return;
+            }
+            if (active) {
+                const uint8_t* st = stage0 + (size_t)s * L.bytes;
+                const uint8_t* wt = st + warp * TILE_BYTES + lane * 16;
+                uint32_t lo[F::NLO], hi[F::NHI];
+#pragma unroll
+                for (int i = 0; i < G::W0; i++) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(wt + i * 512);
+                    lo[4 * i] = v.x; lo[4 * i + 1] = v.y; lo[4 * i + 2] = v.z; lo[4 * i + 3] = v.w;
+                }
+#pragma unroll
+                for (int i = 0; i < G::W1; i++) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(wt + 512 * G::W0 + i * 512);
+                    hi[4 * i] = v.x; hi[4 * i + 1] = v.y; hi[4 * i + 2] = v.z; hi[4 * i + 3] = v.w;
+                }
+                if constexpr (G::W1 == 0) hi[0] = 0;
+                // B-fragment source rows: plane 8*nb + g (token (8*nb + g)/2, hi or lo)
+                const uint8_t* prow[NB];
+                bool pval[NB];
+                float sc2[NB];
+#pragma unroll
+                for (int nb = 0; nb < NB; nb++) {
+                    const int pl = 8 * nb + g;
+                    pval[nb] = pl < 2 * M;
+                    prow[nb] = st + L.planes + (pval[nb] ? pl : 0) * kPlanePitch + 8 * c;
+                    const int tok = 4 * nb + c;
+                    sc2[nb] = tok < M ? ldexpf(1.0f, reinterpret_cast<const int*>(st + L.expo)[tok]) : 0.0f;
+                }
+                const uint16_t* ss = reinterpret_cast<const uint16_t*>(st + L.sc);
+                const uint16_t* zz = reinterpret_cast<const uint16_t*>(st + L.zr);
+                const int* xs = reinterpret_cast<const int*>(st + L.xsum);
+                const int jb = (int)((kc * kChunk) / GROUP) & 7;
+                int ci[NB][4];
+                static_for<0, 8>([&](auto kap_c) {
+                    constexpr int kap = decltype(kap_c)::value;
+                    const uint32_t a0 = F::template reg<kap, 0, 0>(lo, hi);
+                    const uint32_t a1 = F::template reg<kap, 1, 0>(lo, hi);
+                    const uint32_t a2 = F::template reg<kap, 0, 1>(lo, hi);
+                    const uint32_t a3 = F::template reg<kap, 1, 1>(lo, hi);
+#pragma unroll
+                    for (int nb = 0; nb < NB; nb++) {
+                        uint2 bv = make_uint2(0u, 0u);
+                        if (pval[nb]) bv = *reinterpret_cast<const uint2*>(prow[nb] + 32 * kap);
+                        if constexpr (kap % KPG == 0) {
+                            ci[nb][0] = ci[nb][1] = ci[nb][2] = ci[nb][3] = 0;
+                        }
+                        mma_16832_u8s8(ci[nb], a0, a1, a2, a3, bv.x, bv.y);
+                    }
+                    if constexpr (kap % KPG == KPG - 1) {
+                        constexpr int gi = kap / KPG;
+                        const int jj = jb + gi;
+                        const float sg = __half2float(__ushort_as_half(ss[rl * kScaleBox + jj]));
+                        const float sg8 = __half2float(__ushort_as_half(ss[(rl + 8) * kScaleBox + jj]));
+                        const int zg = __half2int_rn(__ushort_as_half(zz[rl * kScaleBox + jj]));
+                        const int zg8 = __half2int_rn(__ushort_as_half(zz[(rl + 8) * kScaleBox + jj]));
+#pragma unroll
+                        for (int nb = 0; nb < NB; nb++) {
+                            const int tok = 4 * nb + c;
+                            const int X = tok < M ? xs[tok * 8 + gi] : 0;
+                            const int S0 = 256 * ci[nb][0] + ci[nb][1] - zg * X;
+                            const int S1 = 256 * ci[nb][2] + ci[nb][3] - zg8 * X;
+                            acc[nb][0] = fmaf(sg * sc2[nb], (float)S0, acc[nb][0]);
+                            acc[nb][1] = fmaf(sg8 * sc2[nb], (float)S1, acc[nb][1]);
+                        }
+                    }
+                });
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty(s));
+        }
+        if (active)
+            tile_epilogue<NB>(acc, (kc0 == 0) && (kc1 == KCH), M, n, tile, rb, KCH, S_total, NC, blockIdx.x,
+                              partials, counters, maxc, y);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+// [rows x cols] fp16 array, box of 128 rows x kScaleBox columns, zero fill outside.
+static bool encode_scale_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+    cuuint32_t box[2] = {kScaleBox, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int gemv_nstage(int bits, int M) {
+    const int sb = StageLayout(bits, M).bytes;
+    const int ns = (kGemvSmemBudget - kBarBytes) / sb;
+    return ns > 12 ? 12 : ns;
+}
+
+bool gemv_group_tma_supported(int64_t M, int64_t n, int64_t k, int bits, int group) {
+    if (M < 1 || M > 16 || k % kChunk != 0 || n % 16 != 0 || bits < 2 || bits > 6) return false;
+    if ((k / group) % 8 != 0) return false;              // 16-byte row stride of the scale arrays
+    if (n > ((int64_t)1 << 31) || k / group > ((int64_t)1 << 31)) return false;
+    return gemv_nstage(bits, (int)M) >= 2;
+}
+
+struct GemvGrid {
+    int grid, maxc;
+};
+static GemvGrid gemv_grid(int64_t n, int64_t k) {
+    const int64_t n_tiles = n / 16;
+    const int64_t n_rb = ceil_div(n_tiles, kConsumers);
+    const int64_t S_total = n_rb * (k / kChunk);
+    GemvGrid gg;
+    gg.grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sm_count() * 2, S_total));
+    gg.maxc = (int)(gg.grid / std::max<int64_t>(n_rb, 1) + 2);
+    return gg;
+}
+
+size_t gemv_group_tma_ws_bytes(int64_t M, int64_t n, int64_t k) {
+    const GemvGrid gg = gemv_grid(n, k);
+    return kCounterBytes + (size_t)((n / 16) * gg.maxc * 16 * M * 4);
+}
+
+template <int B, int GROUP, int NB, bool BF16>
+static lbq_status launch_inst(int grid, size_t smem, int nstage, cudaStream_t st, const CUtensorMap& ms,
+                              const CUtensorMap& mz, const uint16_t* x, int M, const uint8_t* packed, int64_t n,
+                              int64_t k, uint16_t* y, float* part, unsigned* cnt, int maxc) {
+    auto kern = k_gemv_group_tc<B, GROUP, NB, BF16>;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvSmemBudget) != cudaSuccess)
+            return LBQ_ERR_CUDA;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kGemvThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    unsigned* errw = device_error_word();
+    if (cudaLaunchKernelEx(&cfg, kern, ms, mz, x, M, packed, n, k, y, part, cnt, maxc, nstage, errw) != cudaSuccess)
+        return LBQ_ERR_CUDA;
+    return launch_status();
+}
+
+template <int B, bool BF16>
+static lbq_status launch_b(int group, int NB, int grid, size_t smem, int nstage, cudaStream_t st,
+                           const CUtensorMap& ms, const CUtensorMap& mz, const uint16_t* x, int M,
+                           const uint8_t* packed, int64_t n, int64_t k, uint16_t* y, float* part, unsigned* cnt,
+                           int maxc) {
+#define LBQ_I(GR, NBV) launch_inst<B, GR, NBV, BF16>(grid, smem, nstage, st, ms, mz, x, M, packed, n, k, y, part, cnt, maxc)
+#define LBQ_NB(GR) (NB == 1 ? LBQ_I(GR, 1) : NB == 2 ? LBQ_I(GR, 2) : NB == 3 ? LBQ_I(GR, 3) : LBQ_I(GR, 4))
+    if (group == 32) return LBQ_NB(32);
+    if (group == 64) return LBQ_NB(64);
+    return LBQ_NB(128);
+#undef LBQ_NB
+#undef LBQ_I
+}
+
+lbq_status launch_gemv_group_tma(const void* x, bool bf16, int64_t M, const void* packed, const void* scales,
+                                 const void* zeros, int64_t n, int64_t k, int bits, int group, void* y, void* ws,
+                                 size_t ws_bytes, cudaStream_t st) {
+    const GemvGrid gg = gemv_grid(n, k);
+    if (ws == nullptr || ws_bytes < gemv_group_tma_ws_bytes(M, n, k)) return LBQ_ERR_WORKSPACE;
+    if (encode_fn() == nullptr) return LBQ_ERR_CUDA;
+    CUtensorMap ms, mz;
+    if (!encode_scale_map(&ms, scales, n, k / group) || !encode_scale_map(&mz, zeros, n, k / group))
+        return LBQ_ERR_CUDA;
+    const int nstage = gemv_nstage(bits, (int)M);
+    const size_t smem = kBarBytes + (size_t)nstage * StageLayout(bits, (int)M).bytes;
+    const int NB = (int)((2 * M + 7) / 8);
+    auto* cnt = (unsigned*)ws;
+    auto* part = (float*)((char*)ws + kCounterBytes);
+    auto* xp = (const uint16_t*)x;
+    auto* pp = (const uint8_t*)packed;
+    auto* yp = (uint16_t*)y;
+#define LBQ_TB(BB, BF) launch_b<BB, BF>(group, NB, gg.grid, smem, nstage, st, ms, mz, xp, (int)M, pp, n, k, yp, part, cnt, gg.maxc)
+    if (bf16) {
+        switch (bits) {
+            case 2: return LBQ_TB(2, true);
+            case 3: return LBQ_TB(3, true);
+            case 4: return LBQ_TB(4, true);
+            case 5: return LBQ_TB(5, true);
+            default: return LBQ_TB(6, true);
+        }
+    }
+    switch (bits) {
+        case 2: return LBQ_TB(2, false);
+        case 3: return LBQ_TB(3, false);
+        case 4: return LBQ_TB(4, false);
+        case 5: return LBQ_TB(5, false);
+        default: return LBQ_TB(6, false);
+    }
+#undef LBQ_TB
+}
+
+}  // namespace lbq

@@ -12,32 +12,23 @@ int sm_count();
 
 // Geometry of the fragment-interleaved group-code layout (LBQ_LAYOUT_KERNEL).
 // A b-bit code is a low plane of W0 bits and a high plane of W1 = b - W0 bits.
-// Blocks of 512 bytes hold 16 rows x 256/w codes of one plane; a superblock of
-// SB = 256 / min(W0, W1) codes along k holds NB0 = SB*W0/256 low blocks then
-// NB1 = SB*W1/256 high blocks (SB_BYTES = 2*SB*b).
+// Rows come in tiles of 16 and k in superblocks of 256; one (tile, superblock)
+// holds 512*b bytes: the low plane (W0 chunks of 512 B) then the high plane
+// (W1 chunks).  In a plane of width w each 32-bit word holds O = 4/w "octets"
+// (8 consecutive codes of one row) so that byte-masking the word yields the
+// m16n8k32 u8 A-fragment registers of one lane.
 template <int B>
 struct GroupGeom {
     static constexpr int W0 = (B == 2 || B == 3) ? 2 : 4;
     static constexpr int W1 = B - W0;
-    static constexpr int WMIN = (W1 > 0 && W1 < W0) ? W1 : W0;
-    static constexpr int SB = 256 / WMIN;
-    static constexpr int NB0 = SB * W0 / 256;
-    static constexpr int NB1 = SB * W1 / 256;
+    static constexpr int SB = 256;
+    static constexpr int NB0 = W0;          // 512-byte chunks of the low plane
+    static constexpr int NB1 = W1;
     static constexpr int NBLK = NB0 + NB1;
-    static constexpr int SB_BYTES = 2 * SB * B;
-    static_assert(NBLK * 512 == SB_BYTES, "layout geometry");
+    static constexpr int SB_BYTES = 512 * B;
 };
 
-inline int64_t group_superblock(int bits) {
-    switch (bits) {
-        case 2: return GroupGeom<2>::SB;
-        case 3: return GroupGeom<3>::SB;
-        case 4: return GroupGeom<4>::SB;
-        case 5: return GroupGeom<5>::SB;
-        case 6: return GroupGeom<6>::SB;
-        default: return 0;
-    }
-}
+inline int64_t group_superblock(int bits) { return (bits >= 2 && bits <= 6) ? 256 : 0; }
 
 inline int64_t sign_cols_pad(int64_t cols) { return (cols + 255) / 256 * 256; }
 
@@ -58,10 +49,17 @@ lbq_status launch_pack_signs(const int8_t* pm1, int64_t rows, int64_t cols, lbq_
 lbq_status launch_repack_signs(const uint32_t* canon, int64_t rows, int64_t cols, void* out, cudaStream_t st);
 
 // Group GEMV (M <= 16).  ws layout and size: gemv_group_ws_bytes.
-size_t gemv_group_ws_bytes(int64_t M, int64_t n, int64_t k, int bits, lbq_layout layout);
+size_t gemv_group_ws_bytes(int64_t M, int64_t n, int64_t k, int bits, int group, lbq_layout layout);
 lbq_status launch_gemv_group(const void* x, bool bf16, int64_t M, const void* packed, const void* scales,
                              const void* zeros, int64_t n, int64_t k, int bits, int group, lbq_layout layout,
                              void* y, void* ws, size_t ws_bytes, cudaStream_t st);
+
+// TMA-pipelined group GEMV (kernel layout, M <= 16, k % 256 == 0, (k/group) % 8 == 0).
+bool gemv_group_tma_supported(int64_t M, int64_t n, int64_t k, int bits, int group);
+size_t gemv_group_tma_ws_bytes(int64_t M, int64_t n, int64_t k);
+lbq_status launch_gemv_group_tma(const void* x, bool bf16, int64_t M, const void* packed, const void* scales,
+                                 const void* zeros, int64_t n, int64_t k, int bits, int group, void* y, void* ws,
+                                 size_t ws_bytes, cudaStream_t st);
 
 // Batched group GEMM on tcgen05 (M >= 64, kernel layout).
 size_t gemm_group_tc_ws_bytes(int64_t M, int64_t n, int64_t k);

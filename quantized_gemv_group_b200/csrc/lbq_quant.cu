@@ -129,56 +129,52 @@ __global__ void k_unpack_canonical(const uint32_t* __restrict__ in, int64_t nchu
 }
 
 // ---------------------------------------------------------------- kernel layout
-// Each output 32-bit word gathers its codes.  Word geometry (GroupGeom in lbq_internal.h):
-// superblock (tile T, k-block S) of 2*SB*b bytes; low-plane then high-plane blocks of
-// 512 B; lane L = 4g + c owns 16 B = words W0 (row g), W1 (row g+8) for the first half
-// of the block's slices, W2 (row g), W3 (row g+8) for the second half; the code at
-// half h, position pi of a w-bit word is k = kblk + 16*(sig0 + pi/2) + 2c + 8*(pi%2) + h.
+// Word-centric: each 32-bit output word gathers (or scatters, when unpacking) its
+// codes.  Word of (tile T, superblock S, plane p of width w, chunk i, lane L = 4g+c,
+// word wi): it holds octets eta = O*omega + o (omega = 4i + wi, O = 4/w, o < O);
+// octet eta is row 16T + g + 8*(eta%2), columns 256S + 32*(eta/2) + 8c + nu, and
+// code nu = 2j + e sits at bits 8j + 2w*o + w*e.
 template <int B, bool UNPACK>
 __global__ void k_kernel_layout(const uint8_t* __restrict__ codes_in, uint32_t* __restrict__ words, int64_t n,
                                 int64_t k, uint8_t* __restrict__ codes_out) {
     using G = GroupGeom<B>;
     const int64_t nwords = n * k * B / 32;
-    const int64_t ksb = k / G::SB;
-    for (int64_t wi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; wi < nwords;
-         wi += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t byte = wi * 4;
+    const int64_t ksb = k / 256;
+    for (int64_t wi_all = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; wi_all < nwords;
+         wi_all += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t byte = wi_all * 4;
         const int64_t sbi = byte / G::SB_BYTES;
         const int64_t T = sbi / ksb, S = sbi % ksb;
         const int off = (int)(byte % G::SB_BYTES);
-        const int blk = off / 512;
-        const int plane = blk < G::NB0 ? 0 : 1;
-        const int beta = plane ? blk - G::NB0 : blk;
+        const int plane = off < 512 * G::W0 ? 0 : 1;
+        const int poff = plane ? off - 512 * G::W0 : off;
         const int w = plane ? G::W1 : G::W0;
-        const int P = 16 / w;
-        const int ib = off % 512;
-        const int L = ib / 16, widx = (ib % 16) / 4;
+        const int O = 4 / w;
+        const int i = poff / 512, L = (poff % 512) / 16, wi = (poff % 16) / 4;
         const int g = L / 4, c = L % 4;
-        const int upper = widx & 1, second = widx >> 1;
-        const int64_t row = T * 16 + g + 8 * upper;
-        const int64_t kblk = S * G::SB + (int64_t)beta * (256 / w);
-        const int sig0 = second ? P / 2 : 0;
+        const int omega = 4 * i + wi;
         const uint32_t vmask = (1u << w) - 1;
-        uint32_t word = UNPACK ? words[wi] : 0u;
-        for (int h = 0; h < 2; h++)
-            for (int pi = 0; pi < P; pi++) {
-                const int64_t kk = kblk + 16 * (sig0 + pi / 2) + 2 * c + 8 * (pi % 2) + h;
-                const int sh = 16 * h + w * pi;
+        uint32_t word = UNPACK ? words[wi_all] : 0u;
+        for (int o = 0; o < O; o++) {
+            const int eta = O * omega + o;
+            const int64_t row = T * 16 + g + 8 * (eta % 2);
+            const int64_t kb = S * 256 + 32 * (eta / 2) + 8 * c;
+            for (int nu = 0; nu < 8; nu++) {
+                const int sh = 8 * (nu / 2) + 2 * w * o + w * (nu % 2);
+                uint8_t* dst = codes_out ? codes_out + row * k + kb + nu : nullptr;
                 if (!UNPACK) {
-                    const uint32_t q = codes_in[row * k + kk];
+                    const uint32_t q = codes_in[row * k + kb + nu];
                     const uint32_t v = plane ? (q >> G::W0) : (q & ((1u << G::W0) - 1));
                     word |= (v & vmask) << sh;
                 } else {
-                    const uint32_t v = (word >> sh) & vmask;
-                    uint8_t* dst = codes_out + row * k + kk;
-                    // the two planes of a code live in different words; each writer owns its bits
-                    if (plane == 0) atomicOr(reinterpret_cast<unsigned*>((uintptr_t)dst & ~(uintptr_t)3),
-                                             v << (8 * ((uintptr_t)dst & 3)));
-                    else atomicOr(reinterpret_cast<unsigned*>((uintptr_t)dst & ~(uintptr_t)3),
-                                  (v << G::W0) << (8 * ((uintptr_t)dst & 3)));
+                    const uint32_t v = ((word >> sh) & vmask) << (plane ? G::W0 : 0);
+                    // low and high planes of a code live in different words: OR into place
+                    atomicOr(reinterpret_cast<unsigned*>((uintptr_t)dst & ~(uintptr_t)3),
+                             v << (8 * ((uintptr_t)dst & 3)));
                 }
             }
-        if (!UNPACK) words[wi] = word;
+        }
+        if (!UNPACK) words[wi_all] = word;
     }
 }
 

@@ -154,6 +154,29 @@ def test_group_gemv_bf16_activations(bits, group):
     assert _rel(_np(y.float()), ref) <= REL_TOL
 
 
+@pytest.mark.parametrize("bits,group,k", [(4, 64, 320), (2, 32, 384), (6, 64, 640), (4, 128, 1152), (3, 32, 96)])
+@pytest.mark.parametrize("M", [1, 12])
+def test_group_gemv_canonical_odd_shapes(bits, group, k, M):
+    """Shapes outside the kernel layout (k not a multiple of 256, or k/group not a
+    multiple of 8) run through the canonical layout; same parity bar."""
+    n = 40
+    W, x, codes, s, z = _group_case(n, k, bits, group, M, seed=k + bits)
+    ref = _oracle_group(x, codes, s, z, n, k, bits, group)
+    y = lbq.lbq_gemv_group(x, lbq.lbq_pack(codes, bits, lbq.LAYOUT_CANONICAL), s, z, n, k, bits, group,
+                           lbq.LAYOUT_CANONICAL)
+    assert _rel(_np(y.float()), ref) <= REL_TOL
+
+
+def test_kernel_layout_rejects_unsupported_scale_stride():
+    # k/group = 2 is not a multiple of 8: the kernel path refuses, launching nothing
+    n, k = 32, 256
+    W, x, codes, s, z = _group_case(n, k, 4, 128, 1, seed=3)
+    packed = lbq.lbq_pack(codes, 4)
+    with pytest.raises(lbq.LbqError) as ei:
+        lbq.lbq_gemv_group(x, packed, s, z, n, k, 4, 128)
+    assert ei.value.status == lbq.ERR_UNSUPPORTED
+
+
 def test_group_gemv_deterministic_and_split_k():
     # n = 1024 (k/v-like): few row blocks, so every block is split across CTAs
     n, k = 1024, 8192

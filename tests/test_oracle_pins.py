@@ -267,9 +267,9 @@ def test_gemv_bf16_activations():
 
 
 def test_single_code_change_moves_one_output_by_closed_form():
-    """Every position of a 16x128 2-bit matrix, in both layouts: raising one code
-    by 1 changes only that row's output, by x[k] * s."""
-    n, k, bits, group = 16, 128, 2, 32
+    """Positions of a 16x256 2-bit matrix, in both layouts: raising one code by 1
+    changes only that row's output, by x[k] * s."""
+    n, k, bits, group = 16, 256, 2, 32
     g = np.random.default_rng(5)
     codes = g.integers(0, 3, (n, k)).astype(np.uint8)          # room for +1
     s = _f16_bits(np.full((n, k // group), 0.5))
@@ -278,7 +278,7 @@ def test_single_code_change_moves_one_output_by_closed_form():
     xv = _f16_val(x)[0]
     for layout in (orc.LAYOUT_CANONICAL, orc.LAYOUT_KERNEL):
         base = orc.gemv_group(x, orc.pack(codes, bits, layout), s, z, n, k, bits, group, layout=layout)
-        for (i, kk) in [(0, 0), (15, 127), (7, 64), (9, 33), (3, 100)]:
+        for (i, kk) in [(0, 0), (15, 255), (7, 64), (9, 33), (3, 100), (12, 201)]:
             c2 = codes.copy()
             c2[i, kk] += 1
             y2 = orc.gemv_group(x, orc.pack(c2, bits, layout), s, z, n, k, bits, group, layout=layout)
