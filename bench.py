@@ -135,16 +135,23 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- workloads
 class BlockWorkload:
-    """Config 1: one 70B decoder block, INT4 g64, batch 1, rotated copies."""
+    """Config 1: one 70B decoder block, INT4 g64, batch 1, rotated copies.
+
+    A step runs the block's seven GEMVs as a decode step would order them: four
+    grouped launches [q,k,v] (one shared input), [o], [gate,up] (one shared input),
+    [down], each a programmatic dependent of the previous one."""
 
     name = "block"
     bits, group, copies = 4, 64, 4
+    LAUNCHES = (("q_proj", "k_proj", "v_proj"), ("o_proj",), ("gate_proj", "up_proj"), ("down_proj",))
 
-    def __init__(self, dev):
+    def __init__(self, dev, M=1):
         from quantized_gemv_group_b200 import lbq
         self.lbq = lbq
         self.dev = dev
+        self.M = M
         self.linears = wl.block_linears()
+        self.by_name = {l.name: i for i, l in enumerate(self.linears)}
         self.sets = []
         for c in range(self.copies):
             layer = []
@@ -153,35 +160,60 @@ class BlockWorkload:
                 codes, s, z = lbq.lbq_quantize_rtn(W, self.bits, self.group)
                 del W
                 packed = lbq.lbq_pack(codes, self.bits, lbq.LAYOUT_KERNEL)
-                layer.append((packed, s, z, codes if c == 0 else None))
+                layer.append((packed, s, z, None))
                 del codes
             self.sets.append(layer)
-        self.x = [synth.activations(1, l.d_in, seed=900 + p, device=dev) for p, l in enumerate(self.linears)]
-        self.y = [torch.empty(1, l.d_out, dtype=torch.float16, device=dev) for l in self.linears]
-        need = max(lbq.lbq_workspace_bytes(lbq.OP_GEMV_GROUP, 1, l.d_out, l.d_in) for l in self.linears)
-        self.ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
-        self.bytes_per_step = sum(wl.gemv_algorithmic_bytes(l.d_out, l.d_in, self.bits, self.group, 1)
-                                  for l in self.linears)
-        self.launches_per_step = len(self.linears)
+        # one input per launch group (shared by q/k/v and by gate/up)
+        self.xg = [synth.activations(M, self.linears[self.by_name[grp[0]]].d_in, seed=900 + gi, device=dev)
+                   for gi, grp in enumerate(self.LAUNCHES)]
+        self.x = [None] * len(self.linears)
+        for gi, grp in enumerate(self.LAUNCHES):
+            for nm in grp:
+                self.x[self.by_name[nm]] = self.xg[gi]
+        self.y = [torch.empty(M, l.d_out, dtype=torch.float16, device=dev) for l in self.linears]
+        need = 256
+        for c in range(self.copies):
+            for grp in self.LAUNCHES:
+                need = max(need, lbq.lbq_gemv_group_multi_workspace_bytes(self._problems(c, grp, self.x), M))
+        self.ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+        self.bytes_per_step = (sum(wl.group_packed_bytes(l.d_out, l.d_in, self.bits, self.group) + 2 * M * l.d_out
+                                   for l in self.linears) + sum(2 * M * x.shape[1] for x in self.xg))
+        self.launches_per_step = len(self.LAUNCHES)
         torch.cuda.synchronize()
+
+    def _problems(self, c, grp, xs):
+        out = []
+        for nm in grp:
+            p = self.by_name[nm]
+            packed, s, z, _ = self.sets[c][p]
+            l = self.linears[p]
+            out.append((xs[p], packed, s, z, self.y[p], l.d_out, l.d_in))
+        return out
 
     def run_copy(self, c, xs=None, ys=None):
         xs = xs or self.x
-        ys = ys or self.y
-        for (packed, s, z, _), l, x, y in zip(self.sets[c], self.linears, xs, ys):
-            self.lbq.lbq_gemv_group(x, packed, s, z, l.d_out, l.d_in, self.bits, self.group,
-                                    self.lbq.LAYOUT_KERNEL, y=y, ws=self.ws)
+        for grp in self.LAUNCHES:
+            self.lbq.lbq_gemv_group_multi(self._problems(c, grp, xs), self.bits, self.group, ws=self.ws)
 
     def config(self):
         return {"workload": "llama2-70b decoder block GEMVs (q,k,v,o,gate,up,down), INT4 RTN g64, batch 1",
                 "shapes": [[l.d_out, l.d_in] for l in self.linears], "bits": self.bits, "group": self.group,
-                "global_batch": 1, "weight_copies_rotated": self.copies,
+                "launches": [list(g) for g in self.LAUNCHES],
+                "global_batch": self.M, "weight_copies_rotated": self.copies,
                 "l2": "inputs larger than L2: 4 rotated weight copies of 481.6 MB each",
                 "parallelism": "replicas"}
 
     def host_inputs(self):
-        return [x.cpu().pin_memory() for x in self.x], [torch.empty_like(y, device="cpu").pin_memory()
-                                                      for y in self.y]
+        return [x.cpu().pin_memory() for x in self.xg], [torch.empty_like(y, device="cpu").pin_memory()
+                                                       for y in self.y]
+
+    def device_inputs(self, xd):
+        """Per-linear input list for the device copies `xd` of the launch-group inputs."""
+        xs = [None] * len(self.linears)
+        for gi, grp in enumerate(self.LAUNCHES):
+            for nm in grp:
+                xs[self.by_name[nm]] = xd[gi]
+        return xs
 
 
 class Sweep80Workload:
@@ -413,12 +445,13 @@ def run_gpu(args, dev):
 
     # end-to-end: the public calls with host buffers, copies inside the timed region
     xh, yh = wk.host_inputs()
-    xd = [torch.empty_like(x) for x in wk.x]
+    xd = [torch.empty_like(x, device=dev) for x in xh]
+    xs_dev = wk.device_inputs(xd) if hasattr(wk, "device_inputs") else xd
     with torch.cuda.stream(stream):
         def e2e_step(i):
             for a, b in zip(xd, xh):
                 a.copy_(b, non_blocking=True)
-            wk.run_copy(i % wk.copies, xs=xd)
+            wk.run_copy(i % wk.copies, xs=xs_dev)
             for a, b in zip(yh, wk.y):
                 a.copy_(b, non_blocking=True)
         for i in range(max(3, args.warmup)):

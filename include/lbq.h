@@ -142,6 +142,32 @@ lbq_status lbq_gemv_group(const void* x, lbq_dtype x_dtype, int64_t M,
                           int64_t n, int64_t k, int bits, int group, lbq_layout layout,
                           void* y, void* ws, size_t ws_bytes, void* stream);
 
+/* One product of a grouped GEMV launch.  All products of one launch share M, the
+ * activation dtype, the bit width and the group size; each has its own shapes. */
+typedef struct {
+    const void* x;        /* [M x k] activations (x_dtype), 16-byte aligned */
+    const void* packed;   /* codes of W [n x k] in LBQ_LAYOUT_KERNEL, 16-byte aligned */
+    const void* scales;   /* [n x k/group] f16, 16-byte aligned */
+    const void* zeros;    /* [n x k/group] f16, 16-byte aligned */
+    void* y;              /* [M x n] f16 output */
+    int64_t n, k;         /* n % 16 == 0, k % 256 == 0, (k/group) % 8 == 0 */
+} lbq_gemv_problem;
+
+#define LBQ_MAX_GEMV_PROBLEMS 8
+
+/* Grouped group GEMV: computes every product of `problems` (1..LBQ_MAX_GEMV_PROBLEMS)
+ * in ONE launch, e.g. the q/k/v or gate/up projections of a decoder block, which
+ * read the same activations (the fused decode step of the dojofullstack page's
+ * "El truco, en un párrafo": a block's layers run one after another, so the GEMVs
+ * that do not depend on each other can share a launch).  Same arithmetic, layout and
+ * error rules as lbq_gemv_group with LBQ_LAYOUT_KERNEL; the launches of one stream
+ * overlap their ramp with the previous kernel's tail, so packed weights, scales and
+ * zeros must not be written by a kernel that signals programmatic completion early.
+ * ws: lbq_gemv_group_multi_workspace_bytes(problems, count, M) bytes. */
+size_t lbq_gemv_group_multi_workspace_bytes(const lbq_gemv_problem* problems, int count, int64_t M);
+lbq_status lbq_gemv_group_multi(const lbq_gemv_problem* problems, int count, lbq_dtype x_dtype, int64_t M,
+                                int bits, int group, void* ws, size_t ws_bytes, void* stream);
+
 /* Same product for any M >= 1 (prefill / batched decode; the batching of the
  * dojofullstack page's "trabajo batch offline" section, where one loaded layer
  * serves many prompts).  M >= 64 with LBQ_LAYOUT_KERNEL uses the tcgen05

@@ -206,6 +206,45 @@ lbq_status lbq_gemv_group(const void* x, lbq_dtype x_dtype, int64_t M, const voi
                              ws_bytes, (cudaStream_t)stream);
 }
 
+static lbq_status check_multi(const lbq_gemv_problem* problems, int count, lbq_dtype x_dtype, int64_t M,
+                              int bits, int group) {
+    if (!problems || count < 1 || count > LBQ_MAX_GEMV_PROBLEMS) return LBQ_ERR_INVALID_ARG;
+    if (M < 0 || M > 16 || (x_dtype != LBQ_F16 && x_dtype != LBQ_BF16)) return LBQ_ERR_INVALID_ARG;
+    int64_t tiles = 0;
+    for (int i = 0; i < count; i++) {
+        const lbq_gemv_problem& p = problems[i];
+        const lbq_status s =
+            check_group_gemv_args(p.x, M, p.packed, p.scales, p.zeros, p.n, p.k, bits, group, LBQ_LAYOUT_KERNEL, p.y);
+        if (s != LBQ_OK) return s;
+        if (M > 0 && p.n > 0 && !gemv_group_tma_supported(M, p.n, p.k, bits, group)) return LBQ_ERR_UNSUPPORTED;
+        tiles += p.n / 16;
+    }
+    return tiles > kMaxTiles ? LBQ_ERR_UNSUPPORTED : LBQ_OK;
+}
+
+size_t lbq_gemv_group_multi_workspace_bytes(const lbq_gemv_problem* problems, int count, int64_t M) {
+    if (!problems || count < 1 || count > LBQ_MAX_GEMV_PROBLEMS || M <= 0) return 0;
+    int64_t n[LBQ_MAX_GEMV_PROBLEMS], k[LBQ_MAX_GEMV_PROBLEMS];
+    for (int i = 0; i < count; i++) {
+        n[i] = problems[i].n;
+        k[i] = problems[i].k;
+    }
+    return gemv_group_tma_ws_bytes_multi(n, k, count, std::min<int64_t>(M, 16));
+}
+
+lbq_status lbq_gemv_group_multi(const lbq_gemv_problem* problems, int count, lbq_dtype x_dtype, int64_t M, int bits,
+                                int group, void* ws, size_t ws_bytes, void* stream) {
+    const lbq_status s = check_multi(problems, count, x_dtype, M, bits, group);
+    if (s != LBQ_OK || M == 0) return s;
+    lbq_gemv_problem live[LBQ_MAX_GEMV_PROBLEMS];
+    int nlive = 0;
+    for (int i = 0; i < count; i++)
+        if (problems[i].n > 0) live[nlive++] = problems[i];
+    if (nlive == 0) return LBQ_OK;
+    return launch_gemv_group_tma_multi(live, nlive, x_dtype == LBQ_BF16, M, bits, group, ws, ws_bytes,
+                                       (cudaStream_t)stream);
+}
+
 lbq_status lbq_gemm_group(const void* x, lbq_dtype x_dtype, int64_t M, const void* packed, const void* scales,
                           const void* zeros, int64_t n, int64_t k, int bits, int group, lbq_layout layout, void* y,
                           void* ws, size_t ws_bytes, void* stream) {

@@ -104,6 +104,16 @@ __device__ __forceinline__ void mma_16832_u8s8(int (&c)[4], uint32_t a0, uint32_
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Same with C = 0 (the first k-step of an accumulation): d = A * B.
+__device__ __forceinline__ void mma_16832_u8s8_zc(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                  uint32_t b0, uint32_t b1) {
+    const int z = 0;
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(z));
+}
+
 // ---------------------------------------------------------------- misc
 // Compile-time loop: f(std::integral_constant<int, I>) for I in [BEGIN, END).
 template <int BEGIN, int END, typename F>

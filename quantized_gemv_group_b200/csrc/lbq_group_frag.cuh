@@ -38,12 +38,13 @@ struct IFrag {
 // 4*nb + c.  If the CTA covered the tile's whole k-range (full) the result is stored
 // directly; otherwise it is written to this CTA's partial slot and the last of the
 // `count` contributing CTAs (atomic ticket) sums the slots in CTA order, stores y and
-// resets the ticket.  Contributors are the CTAs owning the first and last unit of the
-// tile's row block under the even split start(b) = b * S_total / NC.
+// resets the ticket.  The row block's units are [first_u, first_u + units_per_rb) of
+// the launch's unit list, split evenly over NC CTAs (start(b) = b * S_total / NC);
+// `gtile` indexes the launch-wide ticket and partial arrays, `tile` the rows of y.
 template <int NB>
 __device__ __forceinline__ void tile_epilogue(const float (&acc)[NB][2], bool full, int M, int64_t n, int64_t tile,
-                                              int64_t rb, int64_t units_per_rb, int64_t S_total, int64_t NC,
-                                              int64_t cta, float* __restrict__ partials,
+                                              int64_t gtile, int64_t first_u, int64_t units_per_rb, int64_t S_total,
+                                              int64_t NC, int64_t cta, float* __restrict__ partials,
                                               unsigned* __restrict__ counters, int maxc, uint16_t* __restrict__ y) {
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
@@ -59,12 +60,12 @@ __device__ __forceinline__ void tile_epilogue(const float (&acc)[NB][2], bool fu
         }
         return;
     }
-    const int64_t first_u = rb * units_per_rb, last_u = first_u + units_per_rb - 1;
+    const int64_t last_u = first_u + units_per_rb - 1;
     const int64_t own_first = ((first_u + 1) * NC - 1) / S_total;
     const int64_t own_last = ((last_u + 1) * NC - 1) / S_total;
     const int count = (int)(own_last - own_first + 1);
     const int slot = (int)(cta - own_first);
-    float* pslot = partials + ((tile * maxc) + slot) * (int64_t)(16 * M);
+    float* pslot = partials + ((gtile * maxc) + slot) * (int64_t)(16 * M);
 #pragma unroll
     for (int nb = 0; nb < NB; nb++) {
         const int tok = 4 * nb + c;
@@ -77,19 +78,19 @@ __device__ __forceinline__ void tile_epilogue(const float (&acc)[NB][2], bool fu
     unsigned old = 0;
     if (lane == 0) {
         __threadfence();
-        old = atomicAdd(counters + tile, 1u);
+        old = atomicAdd(counters + gtile, 1u);
     }
     old = __shfl_sync(0xffffffffu, old, 0);
     if (old == (unsigned)(count - 1)) {
         __threadfence();
-        const float* p0 = partials + (tile * maxc) * (int64_t)(16 * M);
+        const float* p0 = partials + (gtile * maxc) * (int64_t)(16 * M);
         for (int e = lane; e < 16 * M; e += 32) {
             float s = 0.0f;
             for (int sl = 0; sl < count; sl++) s += __ldcg(p0 + sl * (int64_t)(16 * M) + e);
             y[(int64_t)(e / 16) * n + tile * 16 + (e % 16)] = from_f32<false>(s);
         }
         __syncwarp();
-        if (lane == 0) counters[tile] = 0u;
+        if (lane == 0) counters[gtile] = 0u;
     }
 }
 

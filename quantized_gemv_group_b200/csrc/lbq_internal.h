@@ -36,6 +36,7 @@ inline int64_t sign_cols_pad(int64_t cols) { return (cols + 255) / 256 * 256; }
 // tile, at most kMaxTiles).  It must be zero before the first call; every call
 // leaves it zero.  The bytes after it are scratch, always written before read.
 constexpr int64_t kMaxTiles = 16384;
+constexpr int kMaxGemvProblems = LBQ_MAX_GEMV_PROBLEMS;
 constexpr size_t kCounterBytes = (size_t)kMaxTiles * 4;
 
 lbq_status launch_quantize_rtn(const void* W, bool bf16, int64_t n, int64_t k, int bits, int group,
@@ -57,6 +58,9 @@ lbq_status launch_gemv_group(const void* x, bool bf16, int64_t M, const void* pa
 // TMA-pipelined group GEMV (kernel layout, M <= 16, k % 256 == 0, (k/group) % 8 == 0).
 bool gemv_group_tma_supported(int64_t M, int64_t n, int64_t k, int bits, int group);
 size_t gemv_group_tma_ws_bytes(int64_t M, int64_t n, int64_t k);
+size_t gemv_group_tma_ws_bytes_multi(const int64_t* n, const int64_t* k, int count, int64_t M);
+lbq_status launch_gemv_group_tma_multi(const lbq_gemv_problem* probs, int count, bool bf16, int64_t M, int bits,
+                                       int group, void* ws, size_t ws_bytes, cudaStream_t st);
 lbq_status launch_gemv_group_tma(const void* x, bool bf16, int64_t M, const void* packed, const void* scales,
                                  const void* zeros, int64_t n, int64_t k, int bits, int group, void* y, void* ws,
                                  size_t ws_bytes, cudaStream_t st);

@@ -22,6 +22,15 @@ LAYOUT_CANONICAL, LAYOUT_KERNEL = 0, 1
 OP_GEMV_GROUP, OP_GEMM_GROUP, OP_GEMV_BINLR, OP_GEMM_BINLR = range(4)
 
 
+MAX_GEMV_PROBLEMS = 8
+
+
+class GemvProblem(ctypes.Structure):
+    """lbq_gemv_problem: one product of a grouped GEMV launch."""
+    _fields_ = [("x", ctypes.c_void_p), ("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("zeros", ctypes.c_void_p), ("y", ctypes.c_void_p), ("n", ctypes.c_int64), ("k", ctypes.c_int64)]
+
+
 class LbqError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
@@ -55,6 +64,8 @@ def lib():
             "lbq_gemv_binlr": (i32, [p, i32, i64, p, p, p, p, i64, i64, i64, i32, p, p, sz, p]),
             "lbq_gemm_binlr": (i32, [p, i32, i64, p, p, p, p, i64, i64, i64, i32, p, p, sz, p]),
             "lbq_schedule_bits": (i32, [i32, i32, i32]),
+            "lbq_gemv_group_multi_workspace_bytes": (sz, [p, i32, i64]),
+            "lbq_gemv_group_multi": (i32, [p, i32, i32, i64, i32, i32, p, sz, p]),
             "lbq_last_device_error": (i32, [p, ctypes.POINTER(ctypes.c_int)]),
         }
         for name, (res, args) in sig.items():
@@ -196,6 +207,35 @@ def _group_call(fn, name, op, x, packed, scales, zeros, n, k, bits, group, layou
     _check(fn(_ptr(x), _dtype_code(x), M, _ptr(packed), _ptr(scales), _ptr(zeros), n, k, bits, group, layout,
               _ptr(y), _ptr(ws) if ws.numel() else None, ws.numel(), _stream(stream)), name)
     return y
+
+
+def _problem_array(problems):
+    arr = (GemvProblem * len(problems))()
+    for i, pr in enumerate(problems):
+        x, packed, scales, zeros, y, n, k = pr
+        arr[i] = GemvProblem(_ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), _ptr(y), n, k)
+    return arr
+
+
+def lbq_gemv_group_multi_workspace_bytes(problems, M):
+    arr = _problem_array(problems)
+    return int(lib().lbq_gemv_group_multi_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), len(problems), M))
+
+
+def lbq_gemv_group_multi(problems, bits, group, ws=None, stream=None):
+    """problems: list of (x [M,k], packed, scales, zeros, y [M,n] fp16, n, k) sharing M and x dtype."""
+    if not problems:
+        raise ValueError("no problems")
+    x0 = problems[0][0]
+    M = x0.shape[0] if x0.dim() == 2 else 1
+    arr = _problem_array(problems)
+    need = int(lib().lbq_gemv_group_multi_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), len(problems), M))
+    if ws is None:
+        ws = _ws_for(need, x0.device)
+    _check(lib().lbq_gemv_group_multi(ctypes.cast(arr, ctypes.c_void_p), len(problems), _dtype_code(x0), M, bits,
+                                      group, _ptr(ws) if ws.numel() else None, ws.numel(), _stream(stream)),
+           "lbq_gemv_group_multi")
+    return [pr[4] for pr in problems]
 
 
 def lbq_gemv_group(x, packed, scales, zeros, n, k, bits, group, layout=LAYOUT_KERNEL, y=None, ws=None,

@@ -189,6 +189,40 @@ def test_group_gemv_deterministic_and_split_k():
     assert _rel(_np(y1.float()), ref) <= REL_TOL
 
 
+@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("bits,group", [(4, 64), (2, 32), (5, 32), (3, 128)])
+def test_gemv_group_multi_matches_each_product(M, bits, group):
+    """One grouped launch of heterogeneous products (the q/k/v pattern: shared x,
+    different n; plus a product with its own x and k) equals the oracle per product."""
+    shapes = [(400, 1024), (64, 1024), (64, 1024), (256, 2048)]
+    xa = synth.activations(M, 1024, seed=5, device=DEV)
+    xb = synth.activations(M, 2048, seed=6, device=DEV)
+    probs, refs = [], []
+    for i, (n, k) in enumerate(shapes):
+        W = synth.weight(n, k, seed=50 + i + 10 * bits, device=DEV)
+        codes, s, z = lbq.lbq_quantize_rtn(W, bits, group)
+        x = xa if k == 1024 else xb
+        y = torch.full((M, n), float("nan"), dtype=torch.float16, device=DEV)
+        probs.append((x, lbq.lbq_pack(codes, bits), s, z, y, n, k))
+        refs.append(_oracle_group(x, codes, s, z, n, k, bits, group))
+    lbq.lbq_gemv_group_multi(probs, bits, group)
+    for pr, ref in zip(probs, refs):
+        assert _rel(_np(pr[4].float()), ref) <= REL_TOL
+
+
+def test_gemv_group_multi_argument_errors():
+    x = torch.zeros(1, 256, dtype=torch.float16, device=DEV)
+    codes = torch.zeros(16, 256, dtype=torch.uint8, device=DEV)
+    s = torch.ones(16, 8, dtype=torch.float16, device=DEV)
+    z = torch.zeros(16, 8, dtype=torch.float16, device=DEV)
+    y = torch.empty(1, 16, dtype=torch.float16, device=DEV)
+    pr = (x, lbq.lbq_pack(codes, 4), s, z, y, 16, 256)
+    with pytest.raises(lbq.LbqError):
+        lbq.lbq_gemv_group_multi([pr] * 9, 4, 32)             # more than LBQ_MAX_GEMV_PROBLEMS
+    with pytest.raises(lbq.LbqError):
+        lbq.lbq_gemv_group_multi([pr], 7, 32)                  # bad bit width
+
+
 def test_gemm_group_small_m_blocks():
     n, k, M = 256, 1024, 37                       # 16 + 16 + 5 tokens
     W, x, codes, s, z = _group_case(n, k, 4, 128, M, seed=21, xdtype=torch.bfloat16)
