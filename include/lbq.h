@@ -53,7 +53,8 @@ typedef enum {
     LBQ_ERR_WORKSPACE = 4,     /* workspace missing or smaller than lbq_workspace_bytes() */
     LBQ_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
     LBQ_ERR_TIMEOUT = 6,       /* a bounded device-side wait expired */
-    LBQ_ERR_DEVICE = 7         /* a kernel reported a data error (see lbq_last_device_error) */
+    LBQ_ERR_DEVICE = 7,        /* a kernel reported a data error (see lbq_last_device_error) */
+    LBQ_ERR_SCRATCH_LIMIT = 8  /* the problem needs more scratch than the library's fixed buffer holds */
 } lbq_status;
 
 typedef enum { LBQ_F16 = 0, LBQ_BF16 = 1 } lbq_dtype;
@@ -167,6 +168,23 @@ typedef struct {
 size_t lbq_gemv_group_multi_workspace_bytes(const lbq_gemv_problem* problems, int count, int64_t M);
 lbq_status lbq_gemv_group_multi(const lbq_gemv_problem* problems, int count, lbq_dtype x_dtype, int64_t M,
                                 int bits, int group, void* ws, size_t ws_bytes, void* stream);
+
+/* Group GEMV for callers that cannot allocate device memory where they multiply
+ * (engine plugins handed no workspace, code running after a pool allocator has
+ * reserved all device memory, host callbacks on a stream, where CUDA API calls are not
+ * allowed).  The pages describe no such variant; this is a library convenience.
+ * Same arguments, arithmetic and rules as lbq_gemv_group with LBQ_LAYOUT_KERNEL, but
+ * no workspace: the scratch lives in a fixed 8 MiB device array owned by the library,
+ * which every GPU that loads the library holds until exit.  The first call on each
+ * device looks up the array's address (make that first call before any stream
+ * capture).  Problems needing more scratch than the array holds (lbq_workspace_bytes
+ * of the kernel path above 8 MiB, e.g. M = 16 on very wide layers) return
+ * LBQ_ERR_SCRATCH_LIMIT.  Every call uses the same array, so calls that overlap on the
+ * GPU (other streams, or other host threads) race and must be serialised by the
+ * caller.  It allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+lbq_status lbq_gemv_group_noalloc(const void* x, lbq_dtype x_dtype, int64_t M, const void* packed,
+                                  const void* scales, const void* zeros, int64_t n, int64_t k, int bits,
+                                  int group, void* y, void* stream);
 
 /* Same product for any M >= 1 (prefill / batched decode; the batching of the
  * dojofullstack page's "trabajo batch offline" section, where one loaded layer

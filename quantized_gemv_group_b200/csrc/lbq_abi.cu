@@ -97,6 +97,7 @@ const char* lbq_status_string(lbq_status s) {
         case LBQ_ERR_CUDA: return "CUDA error";
         case LBQ_ERR_TIMEOUT: return "bounded device wait expired";
         case LBQ_ERR_DEVICE: return "kernel reported a data error";
+        case LBQ_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the fixed buffer holds";
     }
     return "unknown status";
 }

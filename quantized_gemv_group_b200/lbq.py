@@ -15,7 +15,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblbq.so")
 
 # lbq_status
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(8)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE, \
+    ERR_SCRATCH_LIMIT = range(9)
 # lbq_dtype / lbq_layout / lbq_op
 F16, BF16 = 0, 1
 LAYOUT_CANONICAL, LAYOUT_KERNEL = 0, 1
@@ -66,6 +67,7 @@ def lib():
             "lbq_schedule_bits": (i32, [i32, i32, i32]),
             "lbq_gemv_group_multi_workspace_bytes": (sz, [p, i32, i64]),
             "lbq_gemv_group_multi": (i32, [p, i32, i32, i64, i32, i32, p, sz, p]),
+            "lbq_gemv_group_noalloc": (i32, [p, i32, i64, p, p, p, i64, i64, i32, i32, p, p]),
             "lbq_last_device_error": (i32, [p, ctypes.POINTER(ctypes.c_int)]),
         }
         for name, (res, args) in sig.items():
@@ -236,6 +238,15 @@ def lbq_gemv_group_multi(problems, bits, group, ws=None, stream=None):
                                       group, _ptr(ws) if ws.numel() else None, ws.numel(), _stream(stream)),
            "lbq_gemv_group_multi")
     return [pr[4] for pr in problems]
+
+
+def lbq_gemv_group_noalloc(x, packed, scales, zeros, n, k, bits, group, y=None, stream=None):
+    """Group GEMV (kernel layout) without a workspace: scratch is the library's fixed array."""
+    M = x.shape[0] if x.dim() == 2 else 1
+    y = y if y is not None else torch.empty(M, n, dtype=torch.float16, device=x.device)
+    _check(lib().lbq_gemv_group_noalloc(_ptr(x), _dtype_code(x), M, _ptr(packed), _ptr(scales), _ptr(zeros), n, k,
+                                        bits, group, _ptr(y), _stream(stream)), "lbq_gemv_group_noalloc")
+    return y
 
 
 def lbq_gemv_group(x, packed, scales, zeros, n, k, bits, group, layout=LAYOUT_KERNEL, y=None, ws=None,

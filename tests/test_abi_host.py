@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(L):
 
 def test_version_and_status_strings(L):
     assert re.match(r"^\d+\.\d+\.\d+$", lbq.version())
-    for s in range(8):
+    for s in range(9):
         assert lbq.status_string(s)
     assert lbq.status_string(0) == "ok"
 
