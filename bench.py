@@ -217,16 +217,21 @@ class BlockWorkload:
 
 
 class Sweep80Workload:
-    """Config 2: 80 layers x 7 linears, mixed bits (attention 5/6, MLP 2/3), g32."""
+    """Config 2: 80 layers x 7 linears, mixed bits (attention 5/6, MLP 2/3), g32, batch 1.
+
+    Each layer runs the decode order [q,k,v] [o] [gate,up] [down] as grouped launches."""
 
     name = "sweep80"
     group, copies = 32, 1
+    LAUNCHES = BlockWorkload.LAUNCHES
 
-    def __init__(self, dev, n_layers=wl.N_LAYERS):
+    def __init__(self, dev, n_layers=wl.N_LAYERS, M=1):
         from quantized_gemv_group_b200 import lbq
         self.lbq = lbq
         self.dev = dev
+        self.M = M
         self.linears = wl.block_linears()
+        self.by_name = {l.name: i for i, l in enumerate(self.linears)}
         self.n_layers = n_layers
         self.layers = []
         for layer in range(n_layers):
@@ -240,34 +245,58 @@ class Sweep80Workload:
                 del codes
                 lw.append((packed, s, z, b))
             self.layers.append(lw)
-        self.x = [synth.activations(1, l.d_in, seed=900 + p, device=dev) for p, l in enumerate(self.linears)]
-        self.y = [torch.empty(1, l.d_out, dtype=torch.float16, device=dev) for l in self.linears]
-        need = max(lbq.lbq_workspace_bytes(lbq.OP_GEMV_GROUP, 1, l.d_out, l.d_in) for l in self.linears)
-        self.ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
-        self.bytes_per_step = sum(
-            wl.gemv_algorithmic_bytes(l.d_out, l.d_in, wl.schedule_bits(ly, l.name, wl.N_LAYERS), self.group, 1)
-            for ly in range(n_layers) for l in self.linears)
-        self.launches_per_step = n_layers * len(self.linears)
+        self.xg = [synth.activations(M, self.linears[self.by_name[grp[0]]].d_in, seed=900 + gi, device=dev)
+                   for gi, grp in enumerate(self.LAUNCHES)]
+        self.x = [None] * len(self.linears)
+        for gi, grp in enumerate(self.LAUNCHES):
+            for nm in grp:
+                self.x[self.by_name[nm]] = self.xg[gi]
+        self.y = [torch.empty(M, l.d_out, dtype=torch.float16, device=dev) for l in self.linears]
+        need = 256
+        for grp in self.LAUNCHES:
+            need = max(need, lbq.lbq_gemv_group_multi_workspace_bytes(self._problems(0, grp, self.x), M))
+        self.ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+        self.bytes_per_step = (sum(
+            wl.group_packed_bytes(l.d_out, l.d_in, wl.schedule_bits(ly, l.name, wl.N_LAYERS), self.group)
+            + 2 * M * l.d_out for ly in range(n_layers) for l in self.linears)
+            + n_layers * sum(2 * M * x.shape[1] for x in self.xg))
+        self.launches_per_step = n_layers * len(self.LAUNCHES)
         torch.cuda.synchronize()
+
+    def _problems(self, layer, grp, xs):
+        out = []
+        for nm in grp:
+            p = self.by_name[nm]
+            packed, s, z, _ = self.layers[layer][p]
+            l = self.linears[p]
+            out.append((xs[p], packed, s, z, self.y[p], l.d_out, l.d_in))
+        return out
 
     def run_copy(self, c, xs=None, ys=None):
         xs = xs or self.x
-        ys = ys or self.y
-        for lw in self.layers:
-            for (packed, s, z, b), l, x, y in zip(lw, self.linears, xs, ys):
-                self.lbq.lbq_gemv_group(x, packed, s, z, l.d_out, l.d_in, b, self.group,
-                                        self.lbq.LAYOUT_KERNEL, y=y, ws=self.ws)
+        for layer in range(self.n_layers):
+            for grp in self.LAUNCHES:
+                b = self.layers[layer][self.by_name[grp[0]]][3]
+                self.lbq.lbq_gemv_group_multi(self._problems(layer, grp, xs), b, self.group, ws=self.ws)
 
     def config(self):
         return {"workload": f"llama2-70b {self.n_layers}-layer decode weight sweep, mixed RTN bits "
                             "(attn 6/5, mlp 3/2), g32, batch 1",
-                "layers": self.n_layers, "group": self.group, "global_batch": 1,
+                "layers": self.n_layers, "group": self.group, "global_batch": self.M,
                 "code_bits_per_weight": wl.schedule_code_bits_per_weight(),
+                "launches": [list(g) for g in self.LAUNCHES],
                 "l2": "inputs larger than L2 (34 GB of packed weights)", "parallelism": "replicas"}
 
     def host_inputs(self):
-        return [x.cpu().pin_memory() for x in self.x], [torch.empty_like(y, device="cpu").pin_memory()
-                                                      for y in self.y]
+        return [x.cpu().pin_memory() for x in self.xg], [torch.empty_like(y, device="cpu").pin_memory()
+                                                       for y in self.y]
+
+    def device_inputs(self, xd):
+        xs = [None] * len(self.linears)
+        for gi, grp in enumerate(self.LAUNCHES):
+            for nm in grp:
+                xs[self.by_name[nm]] = xd[gi]
+        return xs
 
 
 class BinlrWorkload:
