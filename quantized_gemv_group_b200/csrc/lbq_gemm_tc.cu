@@ -1,14 +1,458 @@
-// lbq_gemm_tc.cu -- batched group GEMM on tcgen05 tensor cores (M >= 64).
+// lbq_gemm_tc.cu -- batched group GEMM on tcgen05 tensor cores (sm_100a), M >= 64 tokens.
+//
+//   y[m, i] = sum_k x[m, k] * s[i, k/g] * (q[i, k] - z[i, k/g])
+//
+// With many tokens one loaded weight serves all of them ("AirLLM corre un modelo 70B en
+// una GPU de 4GB...", section "Es genuinamente excelente para trabajo batch offline"),
+// and the product becomes a dense contraction worth the 5th-generation tensor cores.
+// One CTA computes a 128-row x NT-token tile of y^T in tensor memory (TMEM):
+//
+//  * warp 0 streams, with the Tensor Memory Accelerator (TMA), the packed codes of the
+//    eight 16-row tiles for one 256-wide k superblock plus the 128 x 8 scale and zero
+//    boxes into a ring of code stages;
+//  * warp 10 streams the activations x (fp16) in 64-wide k pieces through a 2-D tensor
+//    map with 128-byte swizzle, the K-major layout the tensor core reads;
+//  * warps 2..9 (one per 16-row tile) expand the codes to fp16 weights
+//    w = fp16(s * (q - z)) for the 128 x 64 A piece, K-major with 128-byte swizzle; at
+//    the end they read the fp32 accumulator back from TMEM and store y in fp16;
+//  * warp 1 allocates TMEM and one of its threads issues tcgen05.mma.kind::f16
+//    (M = 128, N = NT, K = 16) from shared-memory descriptors; tcgen05.commit frees the
+//    A and x buffers and finally signals the epilogue.
+// A and B are both fp16 (kind::f16 takes one type for both): bf16 activations are first
+// converted to fp16, exact for values in fp16's normal range.  The weights are rounded
+// to fp16 once (relative error 2^-11 per weight).  Every wait is bounded: on expiry the
+// kernel records kErrTimeout, drains its tensor-core work, frees TMEM and returns.
+#include <cuda.h>
+#include <cstring>
 #include "lbq_common.cuh"
 #include "lbq_internal.h"
 
 namespace lbq {
 
-size_t gemm_group_tc_ws_bytes(int64_t, int64_t, int64_t) { return 0; }
-bool gemm_group_tc_supported(int64_t, int64_t, int64_t, int, int) { return false; }
-lbq_status launch_gemm_group_tc(const void*, bool, int64_t, const void*, const void*, const void*, int64_t, int64_t,
-                                int, int, void*, void*, size_t, cudaStream_t) {
-    return LBQ_ERR_UNSUPPORTED;
+constexpr int kGemmDq = 8;                         // dequant warps, one per 16-row tile
+constexpr int kGemmThreads = (3 + kGemmDq) * 32;   // codes producer, MMA, dequant x8, x producer
+constexpr int kXWarp = 2 + kGemmDq;
+constexpr int kPiece = 64;                         // k per A piece = one 128-byte swizzle row
+constexpr int kCodeStages = 3;
+constexpr int kXStages = 3;
+constexpr int kAStages = 2;
+constexpr int kGScaleBox = 8;                      // groups per scale/zero box
+constexpr int kGScaleTile = 128 * kGScaleBox * 2;  // bytes of one 128 x 8 fp16 box
+constexpr int kAStageBytes = 128 * kPiece * 2;     // 16 KB
+
+struct GemmSmem {
+    int x, a, codes, code_stage, sc, zr, bars, bytes;
+    __host__ __device__ GemmSmem(int B, int NT) {
+        x = 0;                                           // every stage 1024-byte aligned
+        a = x + kXStages * NT * 128;
+        codes = a + kAStages * kAStageBytes;
+        code_stage = 4096 * B + 2 * kGScaleTile;
+        sc = 4096 * B;                                   // offsets inside a code stage
+        zr = sc + kGScaleTile;
+        bars = codes + kCodeStages * code_stage;
+        bytes = bars + 256;
+    }
+};
+
+struct GemmArgs {
+    CUtensorMap mx;        // x (fp16) [M x k], box 64 x NT, 128-byte swizzle
+    CUtensorMap ms, mz;    // scales / zeros [n x k/g] fp16, box 8 x 128
+    const uint8_t* packed;
+    uint16_t* y;
+    int64_t n, k, M;
+    unsigned* err;
+};
+
+// Byte offset of the 16-byte chunk (row r, k-octet k8) in a 128-row x 64-k fp16 piece,
+// K-major with 128-byte swizzle: 8-row atoms of 1024 bytes, chunk index XOR (r mod 8).
+__device__ __forceinline__ uint32_t a_sw128(int r, int k8) {
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((k8 ^ (r & 7)) << 4));
+}
+
+// Half2 holding (1024 + code(j), 1024 + code(j + 2)) for the codes whose low bits sit at
+// bit `sh0` of w0 (bytes j and j+2) and high bits at `sh1` of w1.
+template <int W0, int W1>
+__device__ __forceinline__ uint32_t code_pair_f16(uint32_t w0, uint32_t w1, int sh0, int sh1) {
+    constexpr uint32_t m0 = ((1u << W0) - 1u) * 0x00010001u;
+    uint32_t v = ((w0 >> sh0) & m0) | 0x64006400u;
+    if constexpr (W1 > 0) {
+        constexpr uint32_t m1 = ((1u << W1) - 1u) * 0x00010001u;
+        v |= ((w1 >> sh1) & m1) << W0;
+    }
+    return v;
+}
+
+// Eight consecutive-k weights (one 16-byte A chunk) from one octet of a lane's codes:
+// w0/w1 hold the octet's plane words, o0/o1 its slot inside them.
+template <int W0, int W1>
+__device__ __forceinline__ uint4 dequant_octet(uint32_t w0, uint32_t w1, int o0, int o1, uint32_t zz2, uint32_t ss2) {
+    uint32_t pr[4];
+#pragma unroll
+    for (int jp = 0; jp < 2; jp++) {
+        const uint32_t h0 = code_pair_f16<W0, W1>(w0, w1, 8 * jp + 2 * W0 * o0, 8 * jp + 2 * W1 * o1);
+        const uint32_t h1 = code_pair_f16<W0, W1>(w0, w1, 8 * jp + 2 * W0 * o0 + W0, 8 * jp + 2 * W1 * o1 + W1);
+        pr[jp] = __byte_perm(h0, h1, 0x5410);        // codes 2j, 2j+1 with j = jp
+        pr[jp + 2] = __byte_perm(h0, h1, 0x7632);    // j = jp + 2
+    }
+    uint4 r;
+    uint32_t* rr = &r.x;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        // (1024 + q) - (1024 + z) is exact in fp16; one rounding in the product with s.
+        const __half2 d = __hsub2(*reinterpret_cast<const __half2*>(&pr[j]), *reinterpret_cast<const __half2*>(&zz2));
+        const __half2 w = __hmul2(d, *reinterpret_cast<const __half2*>(&ss2));
+        rr[j] = *reinterpret_cast<const uint32_t*>(&w);
+    }
+    return r;
+}
+
+template <int B, int GROUP, int NT>
+__global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __grid_constant__ GemmArgs a) {
+    using G = GroupGeom<B>;
+    constexpr int W0 = G::W0, W1 = G::W1;
+    constexpr uint32_t kTmemCols = NT < 32 ? 32 : NT;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const GemmSmem S(B, NT);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S.bars);
+    // c_full[3] c_empty[3] x_full[3] x_empty[3] a_full[2] a_empty[2] d_full | tmem address | abort
+    const uint32_t c_full0 = smem_u32(&bars[0]), c_empty0 = smem_u32(&bars[3]);
+    const uint32_t x_full0 = smem_u32(&bars[6]), x_empty0 = smem_u32(&bars[9]);
+    const uint32_t a_full0 = smem_u32(&bars[12]), a_empty0 = smem_u32(&bars[14]);
+    const uint32_t d_full = smem_u32(&bars[16]);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[17]);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[18]);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n_tt = (a.M + NT - 1) / NT;
+    const int64_t rb = blockIdx.x / n_tt, tt = blockIdx.x % n_tt;
+    const int64_t KSB = a.k / 256;
+    const int64_t n_pieces = a.k / kPiece;
+    unsigned* err = a.err;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kCodeStages; i++) {
+            mbar_init(c_full0 + 8 * i, 1);
+            mbar_init(c_empty0 + 8 * i, kGemmDq);
+        }
+        for (int i = 0; i < kXStages; i++) {
+            mbar_init(x_full0 + 8 * i, 1);
+            mbar_init(x_empty0 + 8 * i, 1);
+        }
+        for (int i = 0; i < kAStages; i++) {
+            mbar_init(a_full0 + 8 * i, kGemmDq);
+            mbar_init(a_empty0 + 8 * i, 1);
+        }
+        mbar_init(d_full, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ codes + scales producer
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_first();
+            const int64_t tiles_left = a.n / 16 - rb * 8;
+            const int tiles = (int)(tiles_left < 8 ? tiles_left : 8);
+            for (int64_t sb = 0; sb < KSB && !*abort_flag; sb++) {
+                const int s = (int)(sb % kCodeStages);
+                if (sb >= kCodeStages &&
+                    !mbar_wait_bounded(c_empty0 + 8 * s, (uint32_t)(((sb / kCodeStages) - 1) & 1), err)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                uint8_t* st = smem + S.codes + s * S.code_stage;
+                const uint32_t fb = c_full0 + 8 * s;
+                mbar_arrive_expect_tx(fb, (uint32_t)(tiles * 512 * B + 2 * kGScaleTile));
+                for (int t = 0; t < tiles; t++)
+                    tma_load_1d_hint(smem_u32(st + t * 512 * B),
+                                     a.packed + ((rb * 8 + t) * KSB + sb) * (int64_t)(512 * B), 512 * B, fb, pol);
+                const int j0 = (int)((sb * 256) / GROUP) & ~7;
+                tma_load_2d(smem_u32(st + S.sc), &a.ms, j0, (int)(rb * 128), fb);
+                tma_load_2d(smem_u32(st + S.zr), &a.mz, j0, (int)(rb * 128), fb);
+            }
+        }
+    } else if (warp == kXWarp) {
+        // ------------------------------------------------------------ activation producer
+        if (lane == 0) {
+            for (int64_t p = 0; p < n_pieces && !*abort_flag; p++) {
+                const int xs = (int)(p % kXStages);
+                if (p >= kXStages && !mbar_wait_bounded(x_empty0 + 8 * xs, (uint32_t)(((p / kXStages) - 1) & 1), err)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(x_full0 + 8 * xs, (uint32_t)(NT * 128));
+                tma_load_2d(smem_u32(smem + S.x + xs * NT * 128), &a.mx, (int)(p * kPiece), (int)(tt * NT),
+                            x_full0 + 8 * xs);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            // kind::f16 instruction descriptor: D fp32, A/B fp16, both K-major, N = NT, M = 128.
+            constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+            for (int64_t p = 0; p < n_pieces; p++) {
+                const int as = (int)(p % kAStages), xs = (int)(p % kXStages);
+                if (*abort_flag || !mbar_wait_bounded(a_full0 + 8 * as, (uint32_t)((p / kAStages) & 1), err) ||
+                    !mbar_wait_bounded(x_full0 + 8 * xs, (uint32_t)((p / kXStages) & 1), err)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_base = smem_u32(smem + S.a + as * kAStageBytes);
+                const uint32_t x_base = smem_u32(smem + S.x + xs * NT * 128);
+#pragma unroll
+                for (int kk = 0; kk < kPiece / 16; kk++) {
+                    // 128-byte swizzle, K-major: 8-row atoms 1024 bytes apart; the k step of
+                    // 16 fp16 advances the start address by 32 bytes inside the atom.
+                    const uint64_t da = umma_smem_desc(a_base + kk * 32, 16, 1024, 2);
+                    const uint64_t dx = umma_smem_desc(x_base + kk * 32, 16, 1024, 2);
+                    umma_f16(tmem_d, da, dx, idesc, (p > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(a_empty0 + 8 * as);
+                umma_commit(x_empty0 + 8 * xs);
+            }
+            umma_commit(d_full);
+            // All issued MMAs must finish before TMEM is freed, on the error path too.
+            mbar_wait_bounded(d_full, 0u, err, 1u << 26);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ dequant warps
+        const int T = warp - 2;                         // 16-row tile inside the 128-row block
+        const int g = lane >> 2, c = lane & 3;
+        const int flip = g & 1;                         // store order that keeps 8-lane phases conflict-free
+        constexpr int O0 = 4 / W0;
+        constexpr int O1 = W1 > 0 ? 4 / W1 : 1;
+        for (int64_t sb = 0; sb < KSB && !*abort_flag; sb++) {
+            const int cs = (int)(sb % kCodeStages);
+            if (!mbar_wait_bounded(c_full0 + 8 * cs, (uint32_t)((sb / kCodeStages) & 1), err)) {
+                *abort_flag = 1;
+                break;
+            }
+            const uint8_t* st = smem + S.codes + cs * S.code_stage;
+            const uint8_t* tb = st + T * 512 * B + 16 * lane;
+            const uint16_t* ss = reinterpret_cast<const uint16_t*>(st + S.sc);
+            const uint16_t* zs = reinterpret_cast<const uint16_t*>(st + S.zr);
+            const int jbase = (int)((sb * 256) / GROUP) & ~7;
+            uint4 pl0 = make_uint4(0, 0, 0, 0), pl1 = make_uint4(0, 0, 0, 0);
+            bool ok = true;
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const int64_t p = sb * 4 + q;
+                const int as = (int)(p % kAStages);
+                // Plane words of this lane: octet eta = 4q + 2kl + u lives in word eta / O.
+                if (q % (4 / W0) == 0) pl0 = *reinterpret_cast<const uint4*>(tb + (q / (4 / W0)) * 512);
+                if constexpr (W1 > 0)
+                    if (q % (4 / W1) == 0) pl1 = *reinterpret_cast<const uint4*>(tb + 512 * W0 + (q / (4 / W1)) * 512);
+                if (p >= kAStages &&
+                    !mbar_wait_bounded(a_empty0 + 8 * as, (uint32_t)(((p / kAStages) - 1) & 1), err)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* abuf = smem + S.a + as * kAStageBytes;
+                uint4 out[2][2];
+#pragma unroll
+                for (int kl = 0; kl < 2; kl++) {
+                    const int jj = (int)((sb * 256 + 64 * q + 32 * kl) / GROUP) - jbase;
+#pragma unroll
+                    for (int u = 0; u < 2; u++) {
+                        const int row = 16 * T + g + 8 * u;
+                        const int eta = 4 * q + 2 * kl + u;
+                        const int wi0 = (eta / O0) & 3, o0 = eta % O0;
+                        const uint32_t* p0 = &pl0.x;
+                        const uint32_t* p1 = &pl1.x;
+                        const uint32_t w0 = p0[wi0];
+                        uint32_t w1 = 0;
+                        int o1 = 0;
+                        if constexpr (W1 > 0) {
+                            w1 = p1[(eta / O1) & 3];
+                            o1 = eta % O1;
+                        }
+                        const uint16_t sh = ss[row * kGScaleBox + jj];
+                        const __half zh = __hadd(__ushort_as_half(zs[row * kGScaleBox + jj]), __float2half(1024.f));
+                        const uint32_t zz2 = (uint32_t)__half_as_ushort(zh) * 0x00010001u;
+                        const uint32_t ss2 = (uint32_t)sh * 0x00010001u;
+                        out[u][kl] = dequant_octet<W0, W1>(w0, w1, o0, o1, zz2, ss2);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 2; u++) {
+                    const int row = 16 * T + g + 8 * u;
+#pragma unroll
+                    for (int i = 0; i < 2; i++) {
+                        const int kl = i ^ flip;
+                        const uint4 v = flip ? out[u][i ^ 1] : out[u][i];
+                        *reinterpret_cast<uint4*>(abuf + a_sw128(row, 4 * kl + c)) = v;
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(a_full0 + 8 * as);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                break;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(c_empty0 + 8 * cs);
+        }
+        // ------------------------------------------------------------ epilogue
+        if (mbar_wait_bounded(d_full, 0u, err, 1u << 26) && !*abort_flag) {
+            tc_fence_after();
+            const int quarter = warp & 3;                  // TMEM lanes this warp may access
+            const int half = (warp - 2) >> 2;              // which half of the NT columns
+            const int64_t row = rb * 128 + 32 * quarter + lane;
+#pragma unroll 1
+            for (int c0 = half * (NT / 2); c0 < (half + 1) * (NT / 2); c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(tmem_d + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, v);
+                tmem_wait_ld();
+                if (row < a.n) {
+#pragma unroll
+                    for (int j = 0; j < 16; j++) {
+                        const int64_t tok = tt * NT + c0 + j;
+                        if (tok < a.M) a.y[tok * a.n + row] = from_f32<false>(__uint_as_float(v[j]));
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_d, kTmemCols);
+    }
+}
+
+// bf16 -> fp16 copy of the activations (exact for values in fp16's normal range).
+__global__ void k_bf16_to_f16(const uint16_t* __restrict__ in, uint16_t* __restrict__ out, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        out[i] = __half_as_ushort(__float2half_rn(__uint_as_float((uint32_t)in[i] << 16)));
+}
+
+// ------------------------------------------------------------------ host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn gemm_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+// Row-major [rows x cols] 16-bit matrix, box box_c (inner) x box_r.
+static bool encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_c, uint32_t box_r,
+                      CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = gemm_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+    cuuint32_t box[2] = {box_c, box_r};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Token tile: the smallest of 64 / 128 / 256 that holds M, 256 beyond.
+static int gemm_nt(int64_t M) { return M <= 64 ? 64 : (M <= 128 ? 128 : 256); }
+
+size_t gemm_group_tc_ws_bytes(int64_t M, int64_t n, int64_t k) {
+    (void)n;
+    return kCounterBytes + (size_t)(M * k * 2 + 256);       // fp16 copy of bf16 activations
+}
+
+bool gemm_group_tc_supported(int64_t M, int64_t n, int64_t k, int bits, int group) {
+    if (M < 64 || n % 16 != 0 || k % 256 != 0 || bits < 2 || bits > 6) return false;
+    if (group != 32 && group != 64 && group != 128) return false;
+    if ((k / group) % 8 != 0 || M > ((int64_t)1 << 31) || n > ((int64_t)1 << 31)) return false;
+    return GemmSmem(bits, gemm_nt(M)).bytes + 1024 <= 227 * 1024;
+}
+
+template <int B, int GROUP, int NT>
+static lbq_status launch_gemm_inst(const GemmArgs& args, int64_t grid, size_t smem, cudaStream_t st) {
+    auto kern = k_gemm_group_tc05<B, GROUP, NT>;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LBQ_ERR_CUDA;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return LBQ_ERR_CUDA;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    kern<<<(unsigned)grid, kGemmThreads, smem, st>>>(args);
+    return launch_status();
+}
+
+template <int B, int NT>
+static lbq_status launch_gemm_g(int group, const GemmArgs& args, int64_t grid, size_t smem, cudaStream_t st) {
+    if (group == 32) return launch_gemm_inst<B, 32, NT>(args, grid, smem, st);
+    if (group == 64) return launch_gemm_inst<B, 64, NT>(args, grid, smem, st);
+    return launch_gemm_inst<B, 128, NT>(args, grid, smem, st);
+}
+
+template <int B>
+static lbq_status launch_gemm_b(int group, int NT, const GemmArgs& args, int64_t grid, size_t smem, cudaStream_t st) {
+    if (NT == 64) return launch_gemm_g<B, 64>(group, args, grid, smem, st);
+    if (NT == 128) return launch_gemm_g<B, 128>(group, args, grid, smem, st);
+    return launch_gemm_g<B, 256>(group, args, grid, smem, st);
+}
+
+lbq_status launch_gemm_group_tc(const void* x, bool bf16, int64_t M, const void* packed, const void* scales,
+                                const void* zeros, int64_t n, int64_t k, int bits, int group, void* y, void* ws,
+                                size_t ws_bytes, cudaStream_t st) {
+    if (ws == nullptr || ws_bytes < gemm_group_tc_ws_bytes(M, n, k)) return LBQ_ERR_WORKSPACE;
+    if (gemm_encode_fn() == nullptr) return LBQ_ERR_CUDA;
+    const int NT = gemm_nt(M);
+    const void* xf = x;
+    if (bf16) {
+        uint16_t* conv = (uint16_t*)((char*)ws + kCounterBytes);
+        const int64_t cnt = M * k;
+        const int grid = (int)std::min<int64_t>(ceil_div(cnt, (int64_t)256), (int64_t)sm_count() * 16);
+        k_bf16_to_f16<<<grid, 256, 0, st>>>((const uint16_t*)x, conv, cnt);
+        if (cudaGetLastError() != cudaSuccess) return LBQ_ERR_CUDA;
+        xf = conv;
+    }
+    GemmArgs args;
+    memset(&args, 0, sizeof args);
+    if (!encode_2d(&args.mx, xf, M, k, 64, (uint32_t)NT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&args.ms, scales, n, k / group, kGScaleBox, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_2d(&args.mz, zeros, n, k / group, kGScaleBox, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return LBQ_ERR_CUDA;
+    args.packed = (const uint8_t*)packed;
+    args.y = (uint16_t*)y;
+    args.n = n;
+    args.k = k;
+    args.M = M;
+    args.err = device_error_word();
+    const int64_t grid = ceil_div(n, (int64_t)128) * ceil_div(M, (int64_t)NT);
+    const size_t smem = (size_t)GemmSmem(bits, NT).bytes + 1024;   // + room to align the base to 1024
+    switch (bits) {
+        case 2: return launch_gemm_b<2>(group, NT, args, grid, smem, st);
+        case 3: return launch_gemm_b<3>(group, NT, args, grid, smem, st);
+        case 4: return launch_gemm_b<4>(group, NT, args, grid, smem, st);
+        case 5: return launch_gemm_b<5>(group, NT, args, grid, smem, st);
+        default: return launch_gemm_b<6>(group, NT, args, grid, smem, st);
+    }
 }
 
 }  // namespace lbq

@@ -231,6 +231,40 @@ def test_gemm_group_small_m_blocks():
     assert _rel(_np(y.float()), ref) <= REL_TOL
 
 
+# ---------------------------------------------------------------- batched GEMM on tcgen05 (M >= 64)
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6])
+@pytest.mark.parametrize("group", [32, 64, 128])
+@pytest.mark.parametrize("M", [64, 100, 200, 300])
+def test_gemm_group_tc_sweep(bits, group, M):
+    # 400 rows: three full 128-row blocks and a ragged 16-row block; M = 64 / 100 / 200 / 300
+    # takes token tiles of 64, 128 (ragged), 256 (ragged) and two tiles of 256.
+    n, k = 400, 1024
+    xdtype = torch.bfloat16 if (bits + M) % 2 else torch.float16
+    W, x, codes, s, z = _group_case(n, k, bits, group, M, seed=7 * bits + group + M, xdtype=xdtype)
+    ref = _oracle_group(x, codes, s, z, n, k, bits, group)
+    y = lbq.lbq_gemm_group(x, lbq.lbq_pack(codes, bits), s, z, n, k, bits, group)
+    torch.cuda.synchronize()
+    assert lbq.lbq_last_device_error() == 0
+    assert _rel(_np(y.float()), ref) <= REL_TOL
+    # each output element, not only the aggregate: fp16 weights and fp32 accumulation
+    yf = _np(y.float()).astype(np.float64)
+    scale = np.abs(ref).max()
+    assert np.max(np.abs(yf - ref)) <= 2e-2 * scale
+
+
+def test_gemm_group_tc_deterministic_and_matches_gemv_blocks():
+    n, k, M = 256, 2048, 96
+    W, x, codes, s, z = _group_case(n, k, 4, 64, M, seed=31)
+    packed = lbq.lbq_pack(codes, 4)
+    y1 = lbq.lbq_gemm_group(x, packed, s, z, n, k, 4, 64).clone()
+    y2 = lbq.lbq_gemm_group(x, packed, s, z, n, k, 4, 64).clone()
+    assert torch.equal(y1, y2)
+    # the 16-token GEMV blocks compute the same product
+    yb = torch.cat([lbq.lbq_gemv_group(x[m0:m0 + 16].contiguous(), packed, s, z, n, k, 4, 64)
+                    for m0 in range(0, M, 16)])
+    assert _rel(_np(y1.float()), _np(yb.float()).astype(np.float64)) <= REL_TOL
+
+
 def test_group_gemv_empty_inputs():
     x = torch.zeros(0, 256, dtype=torch.float16, device=DEV)
     codes = torch.zeros(16, 256, dtype=torch.uint8, device=DEV)
@@ -334,6 +368,23 @@ def test_prefill_shapes_int4_g128_bf16_sampled(shape, M):
     packed = lbq.lbq_pack(codes, 4)
     y = lbq.lbq_gemm_group(x, packed, s, z, n, k, 4, 128)
     rows = _sample_rows(n, 32, 5)
+    ref = orc.gemv_group(_u16(x), _np(packed), _u16(s), _u16(z), n, k, 4, 128, layout=orc.LAYOUT_KERNEL,
+                         rows=rows, x_is_bf16=True)
+    assert _rel(_np(y.float())[:, rows], ref) <= REL_TOL
+
+
+@pytest.mark.parametrize("shape", [(28672, 8192), (8192, 28672)], ids=["gate_up", "down"])
+@pytest.mark.parametrize("M", [64, 256, 1024])
+def test_gemm_tc_70b_shapes_int4_g128_bf16_sampled(shape, M):
+    n, k = shape
+    W = synth.weight(n, k, seed=79, device=DEV)
+    x = synth.activations(M, k, seed=80, device=DEV, dtype=torch.bfloat16)
+    codes, s, z = lbq.lbq_quantize_rtn(W, 4, 128)
+    packed = lbq.lbq_pack(codes, 4)
+    y = lbq.lbq_gemm_group(x, packed, s, z, n, k, 4, 128)
+    torch.cuda.synchronize()
+    assert lbq.lbq_last_device_error() == 0
+    rows = _sample_rows(n, 24, 6)
     ref = orc.gemv_group(_u16(x), _np(packed), _u16(s), _u16(z), n, k, 4, 128, layout=orc.LAYOUT_KERNEL,
                          rows=rows, x_is_bf16=True)
     assert _rel(_np(y.float())[:, rows], ref) <= REL_TOL
