@@ -568,13 +568,118 @@ def run_breakdown(args, dev):
                   file=sys.stderr, flush=True)
 
 
+def _tensor_peak():
+    """Dense fp16/bf16 tensor-core TFLOP/s (kind::f16 runs fp16 at the bf16 rate)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def run_prefill(args, dev):
+    """Prefill sweep: gate/up 8192->28672 and down 28672->8192 at M = 1..1024 tokens,
+    INT4 g128 (bf16 activations) and binary low-rank 0.8 bpw.  GEMV kernels below 64
+    tokens, tcgen05 GEMMs from 64.  One JSON line with every case against both the HBM
+    and the tensor-core roofline."""
+    from quantized_gemv_group_b200 import lbq
+    hbm, hbm_kind = _peaks()
+    tc, tc_kind = _tensor_peak()
+    stream = torch.cuda.Stream(device=dev)
+    Ms = [1, 4, 16, 64, 256, 1024]
+    shapes = [("gate_up", 28672, 8192), ("down", 8192, 28672)]
+    reps = 8
+    cases = []
+    for name, n, k in shapes:
+        # INT4 g128: two weight copies (> L2 together) alternate between calls
+        copies = []
+        for c in range(2):
+            W = synth.weight(n, k, seed=synth.tensor_seed(c, 4 if name == "gate_up" else 6), device=dev)
+            codes, s, z = lbq.lbq_quantize_rtn(W, 4, 128)
+            del W
+            copies.append((lbq.lbq_pack(codes, 4), s, z))
+            del codes
+        r = wl.binlr_rank(n, k, 0.8)
+        bcopies = []
+        for c in range(8):
+            seed = 20000 + 10 * c
+            bcopies.append((lbq.lbq_repack_signs(synth.sign_words(n, r, seed, device=dev), n, r),
+                            lbq.lbq_repack_signs(synth.sign_words(r, k, seed + 1, device=dev), r, k),
+                            synth.channel_scales(n, seed + 2, device=dev), synth.channel_scales(k, seed + 3, device=dev)))
+        for M in Ms:
+            x = synth.activations(M, k, seed=31 + M, device=dev, dtype=torch.bfloat16)
+            y = torch.empty(M, n, dtype=torch.float16, device=dev)
+            for fmt in ("int4_g128", "binary_0.8"):
+                if fmt == "int4_g128":
+                    ws = torch.zeros(lbq.lbq_workspace_bytes(lbq.OP_GEMM_GROUP, M, n, k), dtype=torch.uint8, device=dev)
+
+                    def call(i):
+                        pk, s, z = copies[i % 2]
+                        lbq.lbq_gemm_group(x, pk, s, z, n, k, 4, 128, y=y, ws=ws)
+                    byts = wl.gemv_algorithmic_bytes(n, k, 4, 128, M)
+                    flops = 2.0 * M * n * k
+                    path = "tcgen05 GEMM" if M >= 64 else "GEMV (16-token blocks)"
+                else:
+                    ws = torch.zeros(lbq.lbq_workspace_bytes(lbq.OP_GEMM_BINLR, M, n, k, r), dtype=torch.uint8,
+                                     device=dev)
+
+                    def call(i):
+                        U, Vt, s1, s2 = bcopies[i % 8]
+                        lbq.lbq_gemm_binlr(x, U, Vt, s1, s2, n, k, r, lbq.LAYOUT_KERNEL, y=y, ws=ws)
+                    byts = wl.binlr_algorithmic_bytes(n, k, r, M)
+                    flops = 2.0 * M * r * (n + k)
+                    path = "tcgen05 GEMM x2" if M >= 64 else "GEMV (16-token blocks)"
+                with torch.cuda.stream(stream):
+                    for i in range(8):
+                        call(i)
+                    torch.cuda.synchronize()
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=stream):
+                        for i in range(reps):
+                            call(i)
+                    for _ in range(3):
+                        g.replay()
+                    torch.cuda.synchronize()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    R = 5
+                    e0.record(stream)
+                    for _ in range(R):
+                        g.replay()
+                    e1.record(stream)
+                    torch.cuda.synchronize()
+                us = e0.elapsed_time(e1) * 1e3 / (R * reps)
+                t_hbm, t_tc = byts / (hbm * 1e3), flops / (tc * 1e6)
+                bound = "hbm" if t_hbm >= t_tc else "tensor"
+                cases.append({"shape": name, "n": n, "k": k, "M": M, "format": fmt, "path": path,
+                              "us": round(us, 2), "GB_per_s": round(byts / us / 1e3, 1),
+                              "TFLOP_per_s": round(flops / us / 1e6, 1), "bound": bound,
+                              "roofline_frac": round(max(t_hbm, t_tc) / us, 3)})
+                print(f"{name:8s} M={M:5d} {fmt:10s} {us:9.2f} us {byts / us / 1e3:8.1f} GB/s "
+                      f"{flops / us / 1e6:8.1f} TF/s  {bound} frac {max(t_hbm, t_tc) / us:.3f}",
+                      file=sys.stderr, flush=True)
+                del g
+            del x, y
+        del copies, bcopies
+        torch.cuda.empty_cache()
+    line = {"metric": "prefill sweep: us per call and fraction of max(HBM, tensor) roofline",
+            "unit": "us", "n_gpus": 1, "higher_is_better": False, "data": "synthetic",
+            "config": {"workload": "gate/up 8192->28672 and down 28672->8192, M = 1..1024, bf16 activations, "
+                                   "INT4 g128 and binary 0.8 bpw",
+                       "l2": "2 rotated INT4 copies, 8 rotated binary copies"},
+            "peaks": {"hbm_gbs": hbm, "hbm_kind": hbm_kind, "tensor_tflops": tc, "tensor_kind": tc_kind},
+            "cases": cases}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["lbq", "reference"], default="lbq")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="block")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["prefill"], default="block")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="print per-linear device times to stderr and exit")
     args = ap.parse_args()
@@ -585,6 +690,8 @@ def main():
         torch.cuda.set_device(dev)
     if args.breakdown:
         run_breakdown(args, dev)
+    elif args.workload == "prefill":
+        run_prefill(args, dev)
     elif args.impl == "reference":
         run_reference(args, dev)
     else:

@@ -210,7 +210,11 @@ lbq_status lbq_gemv_binlr(const void* x, lbq_dtype x_dtype, int64_t M,
                           int64_t d_out, int64_t d_in, int64_t r, lbq_layout layout,
                           void* y, void* ws, size_t ws_bytes, void* stream);
 
-/* Same for any M >= 1 (blocks of 16 tokens). */
+/* Same for any M >= 1.  M >= 64 with LBQ_LAYOUT_KERNEL runs two tcgen05 GEMMs
+ * (fp16 +-1 signs expanded in shared memory, fp32 accumulation in tensor memory):
+ * t = V^T (s2 ⊙ x) kept in fp16 in the workspace, then y = s1 ⊙ (U t).  Other
+ * cases run the GEMV path over blocks of 16 tokens.
+ * ws: lbq_workspace_bytes(LBQ_OP_GEMM_BINLR, M, d_out, d_in, r) bytes. */
 lbq_status lbq_gemm_binlr(const void* x, lbq_dtype x_dtype, int64_t M,
                           const void* U, const void* Vt, const void* s1, const void* s2,
                           int64_t d_out, int64_t d_in, int64_t r, lbq_layout layout,

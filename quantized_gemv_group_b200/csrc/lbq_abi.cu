@@ -190,8 +190,10 @@ size_t lbq_workspace_bytes(lbq_op op, int64_t M, int64_t n, int64_t k, int64_t r
         case LBQ_OP_GEMV_BINLR:
         case LBQ_OP_GEMM_BINLR: {
             const int64_t m = std::min<int64_t>(M, 16);
-            return std::max(gemv_binlr_ws_bytes(m, n, k, r, LBQ_LAYOUT_KERNEL),
-                            gemv_binlr_ws_bytes(m, n, k, r, LBQ_LAYOUT_CANONICAL));
+            size_t best = std::max(gemv_binlr_ws_bytes(m, n, k, r, LBQ_LAYOUT_KERNEL),
+                                   gemv_binlr_ws_bytes(m, n, k, r, LBQ_LAYOUT_CANONICAL));
+            if (op == LBQ_OP_GEMM_BINLR && M >= 64) best = std::max(best, gemm_binlr_tc_ws_bytes(M, n, k, r));
+            return best;
         }
     }
     return 0;
@@ -283,6 +285,9 @@ lbq_status lbq_gemm_binlr(const void* x, lbq_dtype x_dtype, int64_t M, const voi
     if (x_dtype != LBQ_F16 && x_dtype != LBQ_BF16) return LBQ_ERR_INVALID_ARG;
     const lbq_status s = check_binlr_args(x, M, U, Vt, s1, s2, d_out, d_in, r, layout, y);
     if (s != LBQ_OK || M == 0 || d_out == 0) return s;
+    if (M >= 64 && layout == LBQ_LAYOUT_KERNEL && gemm_binlr_tc_supported(M, d_out, d_in, r))
+        return launch_gemm_binlr_tc(x, x_dtype == LBQ_BF16, M, U, Vt, s1, s2, d_out, d_in, r, y, ws, ws_bytes,
+                                    (cudaStream_t)stream);
     for (int64_t m0 = 0; m0 < M; m0 += 16) {
         const int64_t mb = std::min<int64_t>(16, M - m0);
         const lbq_status st = launch_gemv_binlr((const uint16_t*)x + m0 * d_in, x_dtype == LBQ_BF16, mb, U, Vt, s1,

@@ -1,6 +1,7 @@
-// lbq_gemm_tc.cu -- batched group GEMM on tcgen05 tensor cores (sm_100a), M >= 64 tokens.
+// lbq_gemm_tc.cu -- batched GEMMs on tcgen05 tensor cores (sm_100a), M >= 64 tokens.
 //
-//   y[m, i] = sum_k x[m, k] * s[i, k/g] * (q[i, k] - z[i, k/g])
+//   group codes:  y[m, i] = sum_k x[m, k] * s[i, k/g] * (q[i, k] - z[i, k/g])
+//   +-1 signs:    the two stages of the binary low-rank form (end of this file)
 //
 // With many tokens one loaded weight serves all of them ("AirLLM corre un modelo 70B en
 // una GPU de 4GB...", section "Es genuinamente excelente para trabajo batch offline"),
@@ -40,13 +41,14 @@ constexpr int kGScaleBox = 8;                      // groups per scale/zero box
 constexpr int kGScaleTile = 128 * kGScaleBox * 2;  // bytes of one 128 x 8 fp16 box
 constexpr int kAStageBytes = 128 * kPiece * 2;     // 16 KB
 
+// B = 2..6: group codes with scale/zero boxes; B = 1: a +-1 sign matrix (no scales).
 struct GemmSmem {
     int x, a, codes, code_stage, sc, zr, bars, bytes;
     __host__ __device__ GemmSmem(int B, int NT) {
         x = 0;                                           // every stage 1024-byte aligned
         a = x + kXStages * NT * 128;
         codes = a + kAStages * kAStageBytes;
-        code_stage = 4096 * B + 2 * kGScaleTile;
+        code_stage = 4096 * B + (B > 1 ? 2 * kGScaleTile : 0);
         sc = 4096 * B;                                   // offsets inside a code stage
         zr = sc + kGScaleTile;
         bars = codes + kCodeStages * code_stage;
@@ -55,11 +57,12 @@ struct GemmSmem {
 };
 
 struct GemmArgs {
-    CUtensorMap mx;        // x (fp16) [M x k], box 64 x NT, 128-byte swizzle
-    CUtensorMap ms, mz;    // scales / zeros [n x k/g] fp16, box 8 x 128
-    const uint8_t* packed;
-    uint16_t* y;
-    int64_t n, k, M;
+    CUtensorMap mx;        // B operand (fp16) [M x k], box 64 x NT, 128-byte swizzle
+    CUtensorMap ms, mz;    // scales / zeros [n x k/g] fp16, box 8 x 128 (group codes only)
+    const uint8_t* packed; // A in its kernel layout: 16-row tiles x 256-wide k superblocks
+    const uint16_t* rowscale;  // optional fp16 factor per output row (signs: s1), else null
+    uint16_t* y;           // fp16 [M x ldy]
+    int64_t n, ksb, M, ldy;    // rows of A, k superblocks, tokens, output row stride
     unsigned* err;
 };
 
@@ -106,9 +109,19 @@ __device__ __forceinline__ uint4 dequant_octet(uint32_t w0, uint32_t w1, int o0,
     return r;
 }
 
+// Eight fp16 +-1 values from bit p of each byte of two sign words (bit 1 = +1): byte
+// 0xBC - 0x80 * bit is the high byte of -1.0 / +1.0, and a byte permute places it.
+__device__ __forceinline__ uint4 signs_octet(uint32_t wa, uint32_t wb, int p) {
+    const uint32_t xa = 0xBCBCBCBCu - ((wa >> p) & 0x01010101u) * 0x80u;
+    const uint32_t xb = 0xBCBCBCBCu - ((wb >> p) & 0x01010101u) * 0x80u;
+    return make_uint4(__byte_perm(xa, 0, 0x1404), __byte_perm(xa, 0, 0x3424), __byte_perm(xb, 0, 0x1404),
+                      __byte_perm(xb, 0, 0x3424));
+}
+
 template <int B, int GROUP, int NT>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __grid_constant__ GemmArgs a) {
-    using G = GroupGeom<B>;
+    constexpr bool kSigns = (B == 1);
+    using G = GroupGeom<kSigns ? 4 : B>;
     constexpr int W0 = G::W0, W1 = G::W1;
     constexpr uint32_t kTmemCols = NT < 32 ? 32 : NT;
     extern __shared__ uint8_t smem_raw[];
@@ -126,8 +139,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n_tt = (a.M + NT - 1) / NT;
     const int64_t rb = blockIdx.x / n_tt, tt = blockIdx.x % n_tt;
-    const int64_t KSB = a.k / 256;
-    const int64_t n_pieces = a.k / kPiece;
+    const int64_t KSB = a.ksb;
+    const int64_t n_pieces = KSB * (256 / kPiece);
     unsigned* err = a.err;
 
     if (threadIdx.x == 0) {
@@ -171,13 +184,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
                 }
                 uint8_t* st = smem + S.codes + s * S.code_stage;
                 const uint32_t fb = c_full0 + 8 * s;
-                mbar_arrive_expect_tx(fb, (uint32_t)(tiles * 512 * B + 2 * kGScaleTile));
+                mbar_arrive_expect_tx(fb, (uint32_t)(tiles * 512 * B + (kSigns ? 0 : 2 * kGScaleTile)));
                 for (int t = 0; t < tiles; t++)
                     tma_load_1d_hint(smem_u32(st + t * 512 * B),
                                      a.packed + ((rb * 8 + t) * KSB + sb) * (int64_t)(512 * B), 512 * B, fb, pol);
-                const int j0 = (int)((sb * 256) / GROUP) & ~7;
-                tma_load_2d(smem_u32(st + S.sc), &a.ms, j0, (int)(rb * 128), fb);
-                tma_load_2d(smem_u32(st + S.zr), &a.mz, j0, (int)(rb * 128), fb);
+                if constexpr (!kSigns) {
+                    const int j0 = (int)((sb * 256) / GROUP) & ~7;
+                    tma_load_2d(smem_u32(st + S.sc), &a.ms, j0, (int)(rb * 128), fb);
+                    tma_load_2d(smem_u32(st + S.zr), &a.mz, j0, (int)(rb * 128), fb);
+                }
             }
         }
     } else if (warp == kXWarp) {
@@ -239,6 +254,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
                 break;
             }
             const uint8_t* st = smem + S.codes + cs * S.code_stage;
+            if constexpr (kSigns) {
+                // Sign layout: lane L = 4g + c holds words (row g, cols 4c..4c+3 of each
+                // 32-column block p at bit 8j + p), (row g+8, same), (row g, cols 16 + ...),
+                // (row g+8, cols 16 + ...).  The octet 8c..8c+7 of a block comes from lanes
+                // 4g + 2(c mod 2) and 4g + 2(c mod 2) + 1, word u + 2(c / 2).
+                const uint32_t* tw = reinterpret_cast<const uint32_t*>(st + T * 512);
+                const int la = 4 * g + 2 * (c & 1);
+                uint32_t wa[2], wb[2];
+#pragma unroll
+                for (int u = 0; u < 2; u++) {
+                    wa[u] = tw[4 * la + u + 2 * (c >> 1)];
+                    wb[u] = tw[4 * (la + 1) + u + 2 * (c >> 1)];
+                }
+                bool ok = true;
+#pragma unroll
+                for (int q = 0; q < 4; q++) {
+                    const int64_t p = sb * 4 + q;
+                    const int as = (int)(p % kAStages);
+                    if (p >= kAStages &&
+                        !mbar_wait_bounded(a_empty0 + 8 * as, (uint32_t)(((p / kAStages) - 1) & 1), err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* abuf = smem + S.a + as * kAStageBytes;
+#pragma unroll
+                    for (int u = 0; u < 2; u++) {
+                        const int row = 16 * T + g + 8 * u;
+#pragma unroll
+                        for (int i = 0; i < 2; i++) {
+                            const int kl = i ^ flip;            // 32-column block 2q + kl of the superblock
+                            *reinterpret_cast<uint4*>(abuf + a_sw128(row, 4 * kl + c)) =
+                                signs_octet(wa[u], wb[u], 2 * q + kl);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(a_full0 + 8 * as);
+                }
+                if (!ok) {
+                    *abort_flag = 1;
+                    break;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(c_empty0 + 8 * cs);
+                continue;
+            }
             const uint8_t* tb = st + T * 512 * B + 16 * lane;
             const uint16_t* ss = reinterpret_cast<const uint16_t*>(st + S.sc);
             const uint16_t* zs = reinterpret_cast<const uint16_t*>(st + S.zr);
@@ -311,6 +372,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
             const int quarter = warp & 3;                  // TMEM lanes this warp may access
             const int half = (warp - 2) >> 2;              // which half of the NT columns
             const int64_t row = rb * 128 + 32 * quarter + lane;
+            float rs = 1.0f;
+            if (a.rowscale != nullptr && row < a.n) rs = __half2float(__ushort_as_half(a.rowscale[row]));
 #pragma unroll 1
             for (int c0 = half * (NT / 2); c0 < (half + 1) * (NT / 2); c0 += 16) {
                 uint32_t v[16];
@@ -320,7 +383,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
 #pragma unroll
                     for (int j = 0; j < 16; j++) {
                         const int64_t tok = tt * NT + c0 + j;
-                        if (tok < a.M) a.y[tok * a.n + row] = from_f32<false>(__uint_as_float(v[j]));
+                        if (tok < a.M) a.y[tok * a.ldy + row] = from_f32<false>(__uint_as_float(v[j]) * rs);
                     }
                 }
             }
@@ -334,10 +397,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
     }
 }
 
-// bf16 -> fp16 copy of the activations (exact for values in fp16's normal range).
-__global__ void k_bf16_to_f16(const uint16_t* __restrict__ in, uint16_t* __restrict__ out, int64_t n) {
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        out[i] = __half_as_ushort(__float2half_rn(__uint_as_float((uint32_t)in[i] << 16)));
+// fp16 copy of the activations [M x k], optionally times a per-column fp16 factor
+// (s2 of the binary form).  bf16 -> fp16 alone is exact in fp16's normal range.
+template <bool BF16>
+__global__ void k_to_f16(const uint16_t* __restrict__ in, const uint16_t* __restrict__ colscale, int64_t k,
+                         uint16_t* __restrict__ out, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        float v = to_f32<BF16>(in[i]);
+        if (colscale != nullptr) v *= __half2float(__ushort_as_half(colscale[i % k]));
+        out[i] = __half_as_ushort(__float2half_rn(v));
+    }
+}
+
+static lbq_status to_f16(const void* x, bool bf16, const void* colscale, int64_t M, int64_t k, void* out,
+                         cudaStream_t st) {
+    const int64_t cnt = M * k;
+    const int grid = (int)std::min<int64_t>(ceil_div(cnt, (int64_t)256), (int64_t)sm_count() * 16);
+    if (bf16)
+        k_to_f16<true><<<grid, 256, 0, st>>>((const uint16_t*)x, (const uint16_t*)colscale, k, (uint16_t*)out, cnt);
+    else
+        k_to_f16<false><<<grid, 256, 0, st>>>((const uint16_t*)x, (const uint16_t*)colscale, k, (uint16_t*)out, cnt);
+    return cudaGetLastError() == cudaSuccess ? LBQ_OK : LBQ_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ host side
@@ -359,13 +439,13 @@ static EncodeTiledFn gemm_encode_fn() {
     return fn;
 }
 
-// Row-major [rows x cols] 16-bit matrix, box box_c (inner) x box_r.
-static bool encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_c, uint32_t box_r,
-                      CUtensorMapSwizzle sw) {
+// Row-major [rows x cols] 16-bit matrix with row stride ld elements, box box_c (inner) x box_r.
+static bool encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, uint32_t box_c,
+                      uint32_t box_r, CUtensorMapSwizzle sw) {
     EncodeTiledFn fn = gemm_encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+    cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
     cuuint32_t box[2] = {box_c, box_r};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
@@ -405,13 +485,20 @@ static lbq_status launch_gemm_inst(const GemmArgs& args, int64_t grid, size_t sm
 
 template <int B, int NT>
 static lbq_status launch_gemm_g(int group, const GemmArgs& args, int64_t grid, size_t smem, cudaStream_t st) {
-    if (group == 32) return launch_gemm_inst<B, 32, NT>(args, grid, smem, st);
-    if (group == 64) return launch_gemm_inst<B, 64, NT>(args, grid, smem, st);
-    return launch_gemm_inst<B, 128, NT>(args, grid, smem, st);
+    if constexpr (B == 1) {
+        return launch_gemm_inst<1, 32, NT>(args, grid, smem, st);   // signs: no groups
+    } else {
+        if (group == 32) return launch_gemm_inst<B, 32, NT>(args, grid, smem, st);
+        if (group == 64) return launch_gemm_inst<B, 64, NT>(args, grid, smem, st);
+        return launch_gemm_inst<B, 128, NT>(args, grid, smem, st);
+    }
 }
 
 template <int B>
-static lbq_status launch_gemm_b(int group, int NT, const GemmArgs& args, int64_t grid, size_t smem, cudaStream_t st) {
+static lbq_status launch_gemm_b(int group, const GemmArgs& args, cudaStream_t st) {
+    const int NT = gemm_nt(args.M);
+    const int64_t grid = ceil_div(args.n, (int64_t)128) * ceil_div(args.M, (int64_t)NT);
+    const size_t smem = (size_t)GemmSmem(B, NT).bytes + 1024;   // + room to align the base to 1024
     if (NT == 64) return launch_gemm_g<B, 64>(group, args, grid, smem, st);
     if (NT == 128) return launch_gemm_g<B, 128>(group, args, grid, smem, st);
     return launch_gemm_g<B, 256>(group, args, grid, smem, st);
@@ -422,37 +509,106 @@ lbq_status launch_gemm_group_tc(const void* x, bool bf16, int64_t M, const void*
                                 size_t ws_bytes, cudaStream_t st) {
     if (ws == nullptr || ws_bytes < gemm_group_tc_ws_bytes(M, n, k)) return LBQ_ERR_WORKSPACE;
     if (gemm_encode_fn() == nullptr) return LBQ_ERR_CUDA;
-    const int NT = gemm_nt(M);
     const void* xf = x;
     if (bf16) {
-        uint16_t* conv = (uint16_t*)((char*)ws + kCounterBytes);
-        const int64_t cnt = M * k;
-        const int grid = (int)std::min<int64_t>(ceil_div(cnt, (int64_t)256), (int64_t)sm_count() * 16);
-        k_bf16_to_f16<<<grid, 256, 0, st>>>((const uint16_t*)x, conv, cnt);
-        if (cudaGetLastError() != cudaSuccess) return LBQ_ERR_CUDA;
+        void* conv = (char*)ws + kCounterBytes;
+        const lbq_status s = to_f16(x, true, nullptr, M, k, conv, st);
+        if (s != LBQ_OK) return s;
         xf = conv;
     }
     GemmArgs args;
     memset(&args, 0, sizeof args);
-    if (!encode_2d(&args.mx, xf, M, k, 64, (uint32_t)NT, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&args.ms, scales, n, k / group, kGScaleBox, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_2d(&args.mz, zeros, n, k / group, kGScaleBox, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!encode_2d(&args.mx, xf, M, k, k, 64, (uint32_t)gemm_nt(M), CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&args.ms, scales, n, k / group, k / group, kGScaleBox, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_2d(&args.mz, zeros, n, k / group, k / group, kGScaleBox, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
         return LBQ_ERR_CUDA;
     args.packed = (const uint8_t*)packed;
+    args.rowscale = nullptr;
     args.y = (uint16_t*)y;
     args.n = n;
-    args.k = k;
+    args.ksb = k / 256;
     args.M = M;
+    args.ldy = n;
     args.err = device_error_word();
-    const int64_t grid = ceil_div(n, (int64_t)128) * ceil_div(M, (int64_t)NT);
-    const size_t smem = (size_t)GemmSmem(bits, NT).bytes + 1024;   // + room to align the base to 1024
     switch (bits) {
-        case 2: return launch_gemm_b<2>(group, NT, args, grid, smem, st);
-        case 3: return launch_gemm_b<3>(group, NT, args, grid, smem, st);
-        case 4: return launch_gemm_b<4>(group, NT, args, grid, smem, st);
-        case 5: return launch_gemm_b<5>(group, NT, args, grid, smem, st);
-        default: return launch_gemm_b<6>(group, NT, args, grid, smem, st);
+        case 2: return launch_gemm_b<2>(group, args, st);
+        case 3: return launch_gemm_b<3>(group, args, st);
+        case 4: return launch_gemm_b<4>(group, args, st);
+        case 5: return launch_gemm_b<5>(group, args, st);
+        default: return launch_gemm_b<6>(group, args, st);
     }
+}
+
+// ------------------------------------------------------------------ binary low-rank GEMM
+// y = s1 . U (V^T (s2 . x)) as two tensor-core GEMMs over the sign kernel layout
+// ("70B en 4GB de VRAM: la compresion neural de 2026, es real?", section
+// "1. NanoQuant", bullet "Formulacion"):
+//   stage 1: t[m, j] = sum_i V^T[j, i] * fp16(s2[i] x[m, i])     rows r,     k = d_in
+//   stage 2: y[m, i] = s1[i] * sum_j U[i, j] * t[m, j]           rows d_out, k = r
+// t is kept in fp16 (11-bit significand) between the stages; the sign bits of the
+// 256-column padding are 0 (-1) and meet zero-filled activation columns.
+struct BinGemmWs {
+    uint16_t* xs;      // fp16(s2 . x) [M x d_in]
+    uint16_t* t;       // fp16 [M x ldt]
+    int64_t ldt;
+    size_t bytes;
+};
+
+static BinGemmWs bin_gemm_ws(void* base, int64_t M, int64_t d_in, int64_t r) {
+    BinGemmWs w{};
+    const size_t xs_bytes = ((size_t)(M * d_in * 2) + 255) / 256 * 256;
+    w.ldt = sign_cols_pad(r);
+    w.xs = (uint16_t*)((char*)base + kCounterBytes);
+    w.t = (uint16_t*)((char*)base + kCounterBytes + xs_bytes);
+    w.bytes = kCounterBytes + xs_bytes + (size_t)(M * w.ldt * 2);
+    return w;
+}
+
+size_t gemm_binlr_tc_ws_bytes(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
+    (void)d_out;
+    return bin_gemm_ws(nullptr, M, d_in, r).bytes;
+}
+
+bool gemm_binlr_tc_supported(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
+    if (M < 64 || d_out % 16 != 0 || r % 32 != 0 || d_in % 32 != 0) return false;
+    if (M > ((int64_t)1 << 31) || d_out > ((int64_t)1 << 31) || r > ((int64_t)1 << 31)) return false;
+    return GemmSmem(1, gemm_nt(M)).bytes + 1024 <= 227 * 1024;
+}
+
+lbq_status launch_gemm_binlr_tc(const void* x, bool bf16, int64_t M, const void* U, const void* Vt, const void* s1,
+                                const void* s2, int64_t d_out, int64_t d_in, int64_t r, void* y, void* ws,
+                                size_t ws_bytes, cudaStream_t st) {
+    if (ws == nullptr || ws_bytes < gemm_binlr_tc_ws_bytes(M, d_out, d_in, r)) return LBQ_ERR_WORKSPACE;
+    if (gemm_encode_fn() == nullptr) return LBQ_ERR_CUDA;
+    const BinGemmWs w = bin_gemm_ws(ws, M, d_in, r);
+    lbq_status s = to_f16(x, bf16, s2, M, d_in, w.xs, st);
+    if (s != LBQ_OK) return s;
+    const int NT = gemm_nt(M);
+    GemmArgs a1;
+    memset(&a1, 0, sizeof a1);
+    if (!encode_2d(&a1.mx, w.xs, M, d_in, d_in, 64, (uint32_t)NT, CU_TENSOR_MAP_SWIZZLE_128B)) return LBQ_ERR_CUDA;
+    a1.packed = (const uint8_t*)Vt;
+    a1.rowscale = nullptr;
+    a1.y = w.t;
+    a1.n = r;
+    a1.ksb = sign_cols_pad(d_in) / 256;
+    a1.M = M;
+    a1.ldy = w.ldt;
+    a1.err = device_error_word();
+    s = launch_gemm_b<1>(32, a1, st);
+    if (s != LBQ_OK) return s;
+    GemmArgs a2;
+    memset(&a2, 0, sizeof a2);
+    if (!encode_2d(&a2.mx, w.t, M, r, w.ldt, 64, (uint32_t)NT, CU_TENSOR_MAP_SWIZZLE_128B)) return LBQ_ERR_CUDA;
+    a2.packed = (const uint8_t*)U;
+    a2.rowscale = (const uint16_t*)s1;
+    a2.y = (uint16_t*)y;
+    a2.n = d_out;
+    a2.ksb = sign_cols_pad(r) / 256;
+    a2.M = M;
+    a2.ldy = d_out;
+    a2.err = a1.err;
+    return launch_gemm_b<1>(32, a2, st);
 }
 
 }  // namespace lbq

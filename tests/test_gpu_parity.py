@@ -335,6 +335,40 @@ def test_binlr_deterministic():
     assert torch.equal(y1, y2)
 
 
+@pytest.mark.parametrize("shape", [(400, 288, 96), (256, 1024, 160), (128, 512, 256)],
+                         ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("M", [64, 100, 300])
+def test_gemm_binlr_tc(shape, M):
+    # d_in = 288 and r = 96 / 160 leave 256-column padding in the sign layout; r = 96 and
+    # d_out = 400 leave ragged 128-row blocks; M = 100 / 300 leave ragged token tiles.
+    d_out, d_in, r = shape
+    xdtype = torch.bfloat16 if M == 100 else torch.float16
+    Uw, Vw, s1, s2, x = _binlr_case(d_out, d_in, r, M, seed=d_out + r + M, xdtype=xdtype)
+    y = _binlr_run(Uw, Vw, s1, s2, x, d_out, d_in, r, lbq.LAYOUT_KERNEL, fn=lbq.lbq_gemm_binlr)
+    torch.cuda.synchronize()
+    assert lbq.lbq_last_device_error() == 0
+    ref = _binlr_oracle(Uw, Vw, s1, s2, x, d_out, d_in, r)
+    assert _rel(_np(y.float()), ref) <= REL_TOL
+    # the 16-token GEMV blocks compute the same product
+    yb = torch.cat([_binlr_run(Uw, Vw, s1, s2, x[m0:m0 + 16].contiguous(), d_out, d_in, r, lbq.LAYOUT_KERNEL)
+                    for m0 in range(0, M, 16)])
+    assert _rel(_np(yb.float()), ref) <= REL_TOL
+
+
+def test_gemm_binlr_tc_all_plus_one():
+    # U = V = all +1: y[m, i] = r * s1[i] * sum_k s2[k] x[m, k]
+    d_out, d_in, r, M = 128, 256, 64, 64
+    Uw = torch.full((d_out, r // 32), -1, dtype=torch.int32, device=DEV)
+    Vw = torch.full((r, d_in // 32), -1, dtype=torch.int32, device=DEV)
+    s1 = synth.channel_scales(d_out, 1, device=DEV)
+    s2 = synth.channel_scales(d_in, 2, device=DEV)
+    x = synth.activations(M, d_in, 3, device=DEV)
+    y = _binlr_run(Uw, Vw, s1, s2, x, d_out, d_in, r, lbq.LAYOUT_KERNEL, fn=lbq.lbq_gemm_binlr)
+    xs = _np(x.float()).astype(np.float64) @ _np(s2.float()).astype(np.float64)
+    ref = r * np.outer(xs, _np(s1.float()).astype(np.float64))
+    assert _rel(_np(y.float()), ref) <= REL_TOL
+
+
 # ---------------------------------------------------------------- full 70B shapes, sampled rows
 def _sample_rows(n, count, seed):
     return np.sort(np.random.default_rng(seed).choice(n, size=min(count, n), replace=False))
@@ -387,6 +421,20 @@ def test_gemm_tc_70b_shapes_int4_g128_bf16_sampled(shape, M):
     rows = _sample_rows(n, 24, 6)
     ref = orc.gemv_group(_u16(x), _np(packed), _u16(s), _u16(z), n, k, 4, 128, layout=orc.LAYOUT_KERNEL,
                          rows=rows, x_is_bf16=True)
+    assert _rel(_np(y.float())[:, rows], ref) <= REL_TOL
+
+
+@pytest.mark.parametrize("shape,M", [((28672, 8192), 64), ((28672, 8192), 256), ((8192, 28672), 64)],
+                         ids=["gate_up-64", "gate_up-256", "down-64"])
+def test_gemm_binlr_tc_70b_shapes_sampled(shape, M):
+    d_out, d_in = shape
+    r = wl.binlr_rank(d_out, d_in, 0.8)
+    Uw, Vw, s1, s2, x = _binlr_case(d_out, d_in, r, M, seed=d_out + 3 * d_in, xdtype=torch.bfloat16)
+    y = _binlr_run(Uw, Vw, s1, s2, x, d_out, d_in, r, lbq.LAYOUT_KERNEL, fn=lbq.lbq_gemm_binlr)
+    torch.cuda.synchronize()
+    assert lbq.lbq_last_device_error() == 0
+    rows = _sample_rows(d_out, 32, 4)
+    ref = _binlr_oracle(Uw, Vw, s1, s2, x, d_out, d_in, r, rows=rows)
     assert _rel(_np(y.float())[:, rows], ref) <= REL_TOL
 
 
