@@ -219,7 +219,7 @@ static lbq_status check_multi(const lbq_gemv_problem* problems, int count, lbq_d
         const lbq_status s =
             check_group_gemv_args(p.x, M, p.packed, p.scales, p.zeros, p.n, p.k, bits, group, LBQ_LAYOUT_KERNEL, p.y);
         if (s != LBQ_OK) return s;
-        if (M > 0 && p.n > 0 && !gemv_group_tma_supported(M, p.n, p.k, bits, group)) return LBQ_ERR_UNSUPPORTED;
+        if (M > 0 && p.n > 0 && !gemv_group_ldg_supported(M, p.n, p.k, bits, group)) return LBQ_ERR_UNSUPPORTED;
         tiles += p.n / 16;
     }
     return tiles > kMaxTiles ? LBQ_ERR_UNSUPPORTED : LBQ_OK;
@@ -232,7 +232,7 @@ size_t lbq_gemv_group_multi_workspace_bytes(const lbq_gemv_problem* problems, in
         n[i] = problems[i].n;
         k[i] = problems[i].k;
     }
-    return gemv_group_tma_ws_bytes_multi(n, k, count, std::min<int64_t>(M, 16));
+    return gemv_group_ldg_ws_bytes_multi(n, k, count, std::min<int64_t>(M, 16));
 }
 
 lbq_status lbq_gemv_group_multi(const lbq_gemv_problem* problems, int count, lbq_dtype x_dtype, int64_t M, int bits,
@@ -244,7 +244,7 @@ lbq_status lbq_gemv_group_multi(const lbq_gemv_problem* problems, int count, lbq
     for (int i = 0; i < count; i++)
         if (problems[i].n > 0) live[nlive++] = problems[i];
     if (nlive == 0) return LBQ_OK;
-    return launch_gemv_group_tma_multi(live, nlive, x_dtype == LBQ_BF16, M, bits, group, ws, ws_bytes,
+    return launch_gemv_group_ldg_multi(live, nlive, x_dtype == LBQ_BF16, M, bits, group, ws, ws_bytes,
                                        (cudaStream_t)stream);
 }
 

@@ -187,6 +187,10 @@ __device__ __forceinline__ void tma_load_1d_hint(uint32_t dst, const void* src, 
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
         ::"r"(dst), "l"(src), "r"(bytes), "r"(bar), "l"(policy) : "memory");
 }
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) from global memory into L2.
+__device__ __forceinline__ void l2_prefetch_bulk(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // 2-D tiled tensor copy global -> shared; c0 = innermost coordinate (16-byte aligned in bytes).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int c0, int c1, uint32_t bar) {
     asm volatile(

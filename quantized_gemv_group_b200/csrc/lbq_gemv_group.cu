@@ -10,9 +10,9 @@
 // section "Por qué es lento"), so the kernel streams the packed codes once, at the
 // HBM rate, and does all dequantization in registers.
 //
-// LBQ_LAYOUT_KERNEL runs on integer tensor cores behind a TMA pipeline
-// (lbq_gemv_group_tma.cu).  This file holds the canonical-layout path -- one warp
-// per row, CUDA-core fp32 FMA, any shape with k % 32 == 0 -- and the dispatch.
+// LBQ_LAYOUT_KERNEL runs on integer tensor cores with the weights streamed straight
+// into registers (lbq_gemv_group_ldg.cu).  This file holds the canonical-layout path --
+// one warp per row, CUDA-core fp32 FMA, any shape with k % 32 == 0 -- and the dispatch.
 #include "lbq_common.cuh"
 #include "lbq_internal.h"
 
@@ -75,7 +75,7 @@ k_gemv_group_canonical(const uint16_t* __restrict__ x, int M, const uint32_t* __
 // ------------------------------------------------------------------ host side
 size_t gemv_group_ws_bytes(int64_t M, int64_t n, int64_t k, int bits, int group, lbq_layout layout) {
     if (layout != LBQ_LAYOUT_KERNEL) return 0;
-    if (gemv_group_tma_supported(M, n, k, bits, group)) return gemv_group_tma_ws_bytes(M, n, k);
+    if (gemv_group_ldg_supported(M, n, k, bits, group)) return gemv_group_ldg_ws_bytes(M, n, k);
     return 0;
 }
 
@@ -105,8 +105,8 @@ lbq_status launch_gemv_group(const void* x, bool bf16, int64_t M, const void* pa
         else launch_canonical<false>(bits, grid, st, xp, (int)M, (const uint32_t*)packed, sp, zp, n, k, group, yp);
         return launch_status();
     }
-    if (!gemv_group_tma_supported(M, n, k, bits, group)) return LBQ_ERR_UNSUPPORTED;
-    return launch_gemv_group_tma(x, bf16, M, packed, scales, zeros, n, k, bits, group, y, ws, ws_bytes, st);
+    if (!gemv_group_ldg_supported(M, n, k, bits, group)) return LBQ_ERR_UNSUPPORTED;
+    return launch_gemv_group_ldg(x, bf16, M, packed, scales, zeros, n, k, bits, group, y, ws, ws_bytes, st);
 }
 
 }  // namespace lbq

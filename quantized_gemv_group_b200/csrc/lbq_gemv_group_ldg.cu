@@ -1,0 +1,675 @@
+// lbq_gemv_group_ldg.cu -- dequant-fused group GEMV on integer tensor cores (sm_100a), M = 1..16.
+//
+//   y[m, i] = sum_k x[m, k] * s[i, k/g] * (q[i, k] - z[i, k/g])
+//
+// Decode time per token is the bytes read over the read bandwidth ("AirLLM corre un
+// modelo 70B en una GPU de 4GB...", section "Por qué es lento"), so the packed weights
+// must stream from HBM at full rate while every other cost hides under that stream.
+//
+//  * Work list: the (16-row tile, 256-wide k superblock) units of up to kMaxGemvProblems
+//    products of one bit width and group size (e.g. the q/k/v or gate/up projections of
+//    a decoder block), tile-major.  Every warp of the grid takes an equal contiguous
+//    slice of it ("stream-K" at warp granularity), so all warps finish together; a tile
+//    split between warps is finished by the last one to arrive (tile_epilogue, fixed
+//    order, deterministic).
+//  * Each warp streams its units' packed words straight into registers with 128-bit
+//    non-coherent loads (evict-first in L2), keeping D units in flight: one unit is the
+//    lane's 16 * B bytes of a tile's 512 * B-byte superblock block, already in mma
+//    fragment order.  Warps never wait for one another, so a warp stalled on compute or
+//    on a scale load leaves the other warps' loads in flight.
+//  * A prep kernel turns every distinct activation row into 16-bit fixed point with one
+//    power-of-two scale 2^E per token and 256-wide chunk (|v| <= 32639), stored as two
+//    int8 planes hi, lo (v = 256 hi + lo) in B-fragment order, plus exact per-group sums
+//    of v.  The warps read these through L1.
+//  * Per k-step the lane masks its words into u8 A fragments (one LOP per four codes)
+//    and runs mma.m16n8k32 u8 x s8 -> s32 with the hi and lo planes side by side in N.
+//    Per group the exact integer sum S = sum q v becomes sum (q - z) v = S - z sum(v),
+//    scaled by s into an fp32 chunk accumulator, which is scaled by 2^E once per chunk.
+//  * Both kernels are launched as programmatic dependents: the GEMV's first weight
+//    loads are issued before it waits for the prep kernel (griddepcontrol.wait), and the
+//    prep kernel waits for the previous kernel in the stream before reading x.  Packed
+//    weights, scales and zeros must therefore not be written by a kernel that signals
+//    programmatic completion early.
+// Group codes: "TurboQuant: cuantizar modelos grandes para que quepan en local",
+// section "Compresión por bloques"; RTN codes: "Métodos de cuantización de LLM para
+// ejecutar un modelo de 70B en una sola GPU", section "RTN (Round-To-Nearest)".
+#include <cstring>
+#include "lbq_common.cuh"
+#include "lbq_internal.h"
+#include "lbq_group_frag.cuh"
+
+namespace lbq {
+
+constexpr int kLdgWarps = 8;
+constexpr int kLdgThreads = kLdgWarps * 32;
+constexpr int kLdgChunk = 256;                 // k per unit (one superblock)
+constexpr int kLdgPlaneMax = 32639;            // |v| bound so that (v + 128) >> 8 fits in int8
+
+struct LdgProblem {
+    const uint8_t* packed;
+    const uint16_t* scales;
+    const uint16_t* zeros;
+    uint16_t* y;
+    int64_t n, k, ksb, n_tiles, ngroups, unit_begin, tile_begin;
+    int slot;               // activation prep slot (products that share x share one)
+};
+
+struct LdgArgs {
+    LdgProblem p[kMaxGemvProblems];
+    float* partials;
+    unsigned* counters;
+    int64_t total_units, total_warps;
+    int count, M, maxc;
+};
+
+// Prepared activations of one distinct x: planes [2M][k] (row 2m = hi plane of token m,
+// 2m + 1 = lo plane, B-fragment byte order), exact group sums [M][k / GROUP] and
+// exponents [M][k / 256], in global memory (planes/xsum/expo) or at byte offsets of the
+// CTA's shared memory (sp/sx/se).
+struct PrepSlot {
+    const uint16_t* x;
+    int8_t* planes;
+    float* xsum;
+    int* expo;
+    int64_t k, warp_begin;
+    int sp, sx, se;
+};
+
+struct PrepArgs {
+    PrepSlot s[kMaxGemvProblems];
+    int64_t total_warps;
+    int count, M;
+};
+
+// Smallest E with maxabs * 2^-E <= kLdgPlaneMax (E = 0 for an all-zero chunk), from the
+// exponent and significand fields (maxabs = m * 2^e, m in [1, 2)).
+__device__ __forceinline__ int ldg_fixed_point_exponent(float maxabs) {
+    if (!(maxabs > 0.0f)) return 0;
+    uint32_t u = __float_as_uint(maxabs);
+    int bias = 0;
+    if ((u >> 23) == 0) {                       // subnormal: scale up exactly by 2^64 first
+        u = __float_as_uint(maxabs * 18446744073709551616.0f);
+        bias = 64;
+    }
+    const int e = (int)(u >> 23) - 127 - bias;
+    const float m = __uint_as_float((u & 0x007FFFFFu) | 0x3F800000u);
+    return e - 14 + (m * 16384.0f > (float)kLdgPlaneMax ? 1 : 0);
+}
+
+// 2^p as a float (exact for every p a normal float holds).
+__device__ __forceinline__ float ldg_exp2i(int p) {
+    if (p >= -126 && p <= 127) return __uint_as_float((uint32_t)(p + 127) << 23);
+    return ldexpf(1.0f, p);
+}
+
+// 16 bytes of streamed weights: read once, so no L1 allocation and evict-first in L2.
+__device__ __forceinline__ uint4 ldg_stream(const void* p, uint64_t pol) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+// NG consecutive fp16 values (NG in 2, 4, 8; 2 * NG-byte aligned) through L1.
+template <int NG>
+__device__ __forceinline__ void ldg_halves(const uint16_t* p, uint32_t (&d)[NG / 2]) {
+    if constexpr (NG == 2) {
+        d[0] = __ldg(reinterpret_cast<const unsigned int*>(p));
+    } else if constexpr (NG == 4) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+        d[0] = v.x;
+        d[1] = v.y;
+    } else {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+        d[0] = v.x;
+        d[1] = v.y;
+        d[2] = v.z;
+        d[3] = v.w;
+    }
+}
+
+// ------------------------------------------------------------------ activation prep
+// One warp per (distinct activation row set, token m, 256-wide chunk); lane l holds
+// elements 8l..8l+7 of the chunk and stores them as the B-fragment bytes of k-slots
+// 4(l mod 4).. (even elements) and 16 + 4(l mod 4).. (odd elements) of k-step l / 4.
+// x may have been written by the previous kernel of the stream, so it is read through
+// L2 (ld.global.cg), never through the non-coherent path.
+struct PrepOut {
+    uint2 hi, lo;   // this lane's 8 bytes of the hi and lo planes
+    int gsum;       // exact sum of v over the lane's group (valid on the group's first lane)
+    int E;
+};
+
+template <int GROUP, bool BF16>
+__device__ __forceinline__ PrepOut prep_chunk(const uint16_t* xc, int lane) {
+    const uint4 raw = __ldcg(reinterpret_cast<const uint4*>(xc + 8 * lane));
+    const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+    float v[8];
+    float mx = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 8; e++) {
+        v[e] = to_f32<BF16>((uint16_t)(rw[e / 2] >> (16 * (e & 1))));
+        mx = fmaxf(mx, fabsf(v[e]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    PrepOut r;
+    r.E = ldg_fixed_point_exponent(mx);
+    // v * 2^-E in at most two exact power-of-two multiplications
+    const int e1 = max(-126, min(127, -r.E));
+    const float f1 = ldg_exp2i(e1), f2 = ldg_exp2i(-r.E - e1);
+    uint32_t hev = 0, hod = 0, lev = 0, lod = 0;
+    int sum = 0;
+#pragma unroll
+    for (int e = 0; e < 8; e++) {
+        const int q = __float2int_rn((v[e] * f1) * f2);
+        const int h = (q + 128) >> 8;
+        const int l = q - 256 * h;
+        sum += q;
+        const int sh = 8 * (e >> 1);
+        if (e & 1) {
+            hod |= (uint32_t)(h & 0xFF) << sh;
+            lod |= (uint32_t)(l & 0xFF) << sh;
+        } else {
+            hev |= (uint32_t)(h & 0xFF) << sh;
+            lev |= (uint32_t)(l & 0xFF) << sh;
+        }
+    }
+    constexpr int LPG = GROUP / 8;                 // lanes per group
+#pragma unroll
+    for (int o = 1; o < LPG; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    r.hi = make_uint2(hev, hod);
+    r.lo = make_uint2(lev, lod);
+    r.gsum = sum;                                  // |sum| <= 128 * 32639 < 2^24: exact in fp32
+    return r;
+}
+
+// Warp task wi of the prep list -> (slot, token, chunk).
+__device__ __forceinline__ int prep_task(const PrepArgs& a, int64_t wi, int& m, int64_t& ch) {
+    int s = 0;
+    while (s + 1 < a.count && wi >= a.s[s + 1].warp_begin) s++;
+    const int64_t kch = a.s[s].k / kLdgChunk;
+    const int64_t li = wi - a.s[s].warp_begin;
+    m = (int)(li / kch);
+    ch = li % kch;
+    return s;
+}
+
+// Stand-alone prep into global memory, for activations too large for shared memory.
+template <int GROUP, bool BF16>
+__global__ void __launch_bounds__(256) k_gemv_prep(const __grid_constant__ PrepArgs a) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t wi = ((int64_t)blockIdx.x * 256 + threadIdx.x) >> 5;
+    if (wi >= a.total_warps) return;
+    int m;
+    int64_t ch;
+    const PrepSlot& S = a.s[prep_task(a, wi, m, ch)];
+    const PrepOut r = prep_chunk<GROUP, BF16>(S.x + (int64_t)m * S.k + ch * kLdgChunk, lane);
+    int8_t* row_h = S.planes + (int64_t)(2 * m) * S.k + ch * kLdgChunk;
+    *reinterpret_cast<uint2*>(row_h + 8 * lane) = r.hi;
+    *reinterpret_cast<uint2*>(row_h + S.k + 8 * lane) = r.lo;
+    constexpr int LPG = GROUP / 8;
+    if (lane % LPG == 0) S.xsum[(int64_t)m * (S.k / GROUP) + ch * (kLdgChunk / GROUP) + lane / LPG] = (float)r.gsum;
+    if (lane == 0) S.expo[(int64_t)m * (S.k / kLdgChunk) + ch] = r.E;
+}
+
+// Prepared-activation reads: shared memory (plain loads) or global memory written by the
+// prep kernel of this launch (L2 only: data another grid wrote during this grid's life).
+template <bool SMEMP>
+__device__ __forceinline__ uint2 ld_plane(const int8_t* p) {
+    if constexpr (SMEMP) return *reinterpret_cast<const uint2*>(p);
+    else return __ldcg(reinterpret_cast<const uint2*>(p));
+}
+template <bool SMEMP, class T>
+__device__ __forceinline__ T ld_prep(const T* p) {
+    if constexpr (SMEMP) return *p;
+    else return __ldcg(p);
+}
+
+// ------------------------------------------------------------------ GEMV
+struct LdgCursor {
+    int p;
+    int64_t t, sb;
+};
+
+__device__ __forceinline__ void ldg_advance(const LdgArgs& a, LdgCursor& cu) {
+    if (++cu.sb == a.p[cu.p].ksb) {
+        cu.sb = 0;
+        if (++cu.t == a.p[cu.p].n_tiles) {
+            cu.t = 0;
+            if (cu.p + 1 < a.count) cu.p++;
+        }
+    }
+}
+
+// D units in flight per warp; CPS resident CTAs per SM (2: up to 128 registers a thread);
+// SMEMP: every CTA prepares the activations itself, in its shared memory, right after
+// waiting for the previous kernel (else they come from k_gemv_prep via L2).
+template <int B, int GROUP, int NB, int D, int CPS, bool SMEMP, bool BF16>
+__global__ void __launch_bounds__(kLdgThreads, CPS)
+    k_gemv_group_ldg(const __grid_constant__ LdgArgs a, const __grid_constant__ PrepArgs pa) {
+    using G = GroupGeom<B>;
+    using F = IFrag<B>;
+    constexpr int KPG = GROUP / 32;                // k-steps per group
+    constexpr int NGC = kLdgChunk / GROUP;         // groups per unit
+    constexpr int PF = B == 2 ? 8 : B == 3 ? 5 : B == 4 ? 4 : B == 5 ? 3 : 2;   // units prefetched into L2
+    extern __shared__ __align__(16) uint8_t smem[];
+    griddep_launch_dependents();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int64_t W = a.total_warps, S = a.total_units;
+    const int64_t wid = (int64_t)blockIdx.x * kLdgWarps + warp;
+    // warps past the W that share the list (grid * 8 may exceed it) take no units
+    const int64_t u_begin = wid < W ? wid * S / W : S;
+    const int64_t u_end = wid < W ? (wid + 1) * S / W : S;
+    const int M = a.M;
+    const uint64_t pol = l2_policy_evict_first();
+
+    const bool has_work = u_begin < u_end;
+    LdgCursor cc;
+    cc.p = 0;
+    while (cc.p + 1 < a.count && u_begin >= a.p[cc.p + 1].unit_begin) cc.p++;
+    if (has_work) {
+        const int64_t lu = u_begin - a.p[cc.p].unit_begin;
+        cc.t = lu / a.p[cc.p].ksb;
+        cc.sb = lu % a.p[cc.p].ksb;
+    }
+    LdgCursor lc = cc;
+
+    uint4 wb[D][B];
+    auto load_unit = [&](uint4 (&dst)[B], const LdgCursor& cu) {
+        const LdgProblem& P = a.p[cu.p];
+        const uint8_t* src = P.packed + (cu.t * P.ksb + cu.sb) * (int64_t)(512 * B) + 16 * lane;
+#pragma unroll
+        for (int i = 0; i < B; i++) dst[i] = ldg_stream(src + 512 * i, pol);
+    };
+    // prologue: the first D units' weights (into registers) and the next PF (into L2)
+    // do not depend on the previous kernels
+#pragma unroll
+    for (int d = 0; d < D; d++) {
+        if (u_begin + d < u_end) {
+            load_unit(wb[d], lc);
+            ldg_advance(a, lc);
+        }
+    }
+    if (lane < PF && u_begin + D + lane < u_end) {
+        LdgCursor pc = lc;
+        for (int i = 0; i < lane; i++) ldg_advance(a, pc);
+        const LdgProblem& P = a.p[pc.p];
+        l2_prefetch_bulk(P.packed + (pc.t * P.ksb + pc.sb) * (int64_t)(512 * B), 512 * B);
+    }
+    griddep_wait();
+    if constexpr (SMEMP) {
+        // this CTA's copy of the prepared activations
+        for (int64_t wi = warp; wi < pa.total_warps; wi += kLdgWarps) {
+            int m;
+            int64_t ch;
+            const PrepSlot& Q = pa.s[prep_task(pa, wi, m, ch)];
+            const PrepOut r = prep_chunk<GROUP, BF16>(Q.x + (int64_t)m * Q.k + ch * kLdgChunk, lane);
+            int8_t* row_h = reinterpret_cast<int8_t*>(smem + Q.sp) + (int64_t)(2 * m) * Q.k + ch * kLdgChunk;
+            *reinterpret_cast<uint2*>(row_h + 8 * lane) = r.hi;
+            *reinterpret_cast<uint2*>(row_h + Q.k + 8 * lane) = r.lo;
+            constexpr int LPG = GROUP / 8;
+            if (lane % LPG == 0)
+                reinterpret_cast<float*>(smem + Q.sx)[(int64_t)m * (Q.k / GROUP) + ch * (kLdgChunk / GROUP) +
+                                                      lane / LPG] = (float)r.gsum;
+            if (lane == 0) reinterpret_cast<int*>(smem + Q.se)[(int64_t)m * (Q.k / kLdgChunk) + ch] = r.E;
+        }
+        __syncthreads();
+    }
+    if (!has_work) return;
+
+    float acc[NB][2];
+#pragma unroll
+    for (int nb = 0; nb < NB; nb++) acc[nb][0] = acc[nb][1] = 0.0f;
+    int64_t tile_first_u = u_begin - cc.sb;        // first unit of the tile being accumulated
+
+    for (int64_t base = u_begin; base < u_end; base += D) {
+#pragma unroll
+        for (int d = 0; d < D; d++) {
+            const int64_t u = base + d;
+            if (u < u_end) {
+                const LdgProblem& P = a.p[cc.p];
+                uint32_t lo[F::NLO], hi[F::NHI];
+#pragma unroll
+                for (int i = 0; i < G::W0; i++) {
+                    lo[4 * i] = wb[d][i].x;
+                    lo[4 * i + 1] = wb[d][i].y;
+                    lo[4 * i + 2] = wb[d][i].z;
+                    lo[4 * i + 3] = wb[d][i].w;
+                }
+#pragma unroll
+                for (int i = 0; i < G::W1; i++) {
+                    hi[4 * i] = wb[d][G::W0 + i].x;
+                    hi[4 * i + 1] = wb[d][G::W0 + i].y;
+                    hi[4 * i + 2] = wb[d][G::W0 + i].z;
+                    hi[4 * i + 3] = wb[d][G::W0 + i].w;
+                }
+                if constexpr (G::W1 == 0) hi[0] = 0;
+                // refill this slot with the unit D ahead
+                if (u + D < u_end) {
+                    load_unit(wb[d], lc);
+                    ldg_advance(a, lc);
+                }
+                // scales and zeros of this unit's NGC groups, rows g and g+8
+                const int64_t rl = cc.t * 16 + g;
+                const int64_t j0 = cc.sb * NGC;
+                uint32_t sh0[NGC / 2], sh1[NGC / 2], zh0[NGC / 2], zh1[NGC / 2];
+                ldg_halves<NGC>(P.scales + rl * P.ngroups + j0, sh0);
+                ldg_halves<NGC>(P.scales + (rl + 8) * P.ngroups + j0, sh1);
+                ldg_halves<NGC>(P.zeros + rl * P.ngroups + j0, zh0);
+                ldg_halves<NGC>(P.zeros + (rl + 8) * P.ngroups + j0, zh1);
+                // prepared activations of this product's x
+                const PrepSlot& PS = pa.s[P.slot];
+                const int8_t* planes = SMEMP ? reinterpret_cast<const int8_t*>(smem + PS.sp) : PS.planes;
+                const float* xsum = SMEMP ? reinterpret_cast<const float*>(smem + PS.sx) : PS.xsum;
+                const int* expo = SMEMP ? reinterpret_cast<const int*>(smem + PS.se) : PS.expo;
+                // B-fragment rows: plane 8*nb + g (token (8*nb + g)/2, hi or lo)
+                const int8_t* prow[NB];
+                bool pval[NB];
+#pragma unroll
+                for (int nb = 0; nb < NB; nb++) {
+                    const int pl = 8 * nb + g;
+                    pval[nb] = pl < 2 * M;
+                    prow[nb] = planes + (int64_t)(pval[nb] ? pl : 0) * P.k + cc.sb * kLdgChunk + 8 * c;
+                }
+                float cacc[NB][2];
+#pragma unroll
+                for (int nb = 0; nb < NB; nb++) cacc[nb][0] = cacc[nb][1] = 0.0f;
+                int ci[NB][4];
+                static_for<0, 8>([&](auto kap_c) {
+                    constexpr int kap = decltype(kap_c)::value;
+                    const uint32_t a0 = F::template reg<kap, 0, 0>(lo, hi);
+                    const uint32_t a1 = F::template reg<kap, 1, 0>(lo, hi);
+                    const uint32_t a2 = F::template reg<kap, 0, 1>(lo, hi);
+                    const uint32_t a3 = F::template reg<kap, 1, 1>(lo, hi);
+#pragma unroll
+                    for (int nb = 0; nb < NB; nb++) {
+                        uint2 bv = make_uint2(0u, 0u);
+                        if (pval[nb]) bv = ld_plane<SMEMP>(prow[nb] + 32 * kap);
+                        if constexpr (kap % KPG == 0) mma_16832_u8s8_zc(ci[nb], a0, a1, a2, a3, bv.x, bv.y);
+                        else mma_16832_u8s8(ci[nb], a0, a1, a2, a3, bv.x, bv.y);
+                    }
+                    if constexpr (kap % KPG == KPG - 1) {
+                        constexpr int gi = kap / KPG;
+                        const float sg = __half2float(__ushort_as_half((uint16_t)(sh0[gi / 2] >> (16 * (gi & 1)))));
+                        const float sg8 = __half2float(__ushort_as_half((uint16_t)(sh1[gi / 2] >> (16 * (gi & 1)))));
+                        const float zg = __half2float(__ushort_as_half((uint16_t)(zh0[gi / 2] >> (16 * (gi & 1)))));
+                        const float zg8 = __half2float(__ushort_as_half((uint16_t)(zh1[gi / 2] >> (16 * (gi & 1)))));
+#pragma unroll
+                        for (int nb = 0; nb < NB; nb++) {
+                            const int tok = 4 * nb + c;
+                            const float X = tok < M ? ld_prep<SMEMP>(xsum + tok * P.ngroups + j0 + gi) : 0.0f;
+                            const float f0 = fmaf(-zg, X, (float)(256 * ci[nb][0] + ci[nb][1]));
+                            const float f1 = fmaf(-zg8, X, (float)(256 * ci[nb][2] + ci[nb][3]));
+                            cacc[nb][0] = fmaf(sg, f0, cacc[nb][0]);
+                            cacc[nb][1] = fmaf(sg8, f1, cacc[nb][1]);
+                        }
+                    }
+                });
+#pragma unroll
+                for (int nb = 0; nb < NB; nb++) {
+                    const int tok = 4 * nb + c;
+                    const float sc = tok < M ? ldg_exp2i(ld_prep<SMEMP>(expo + tok * P.ksb + cc.sb)) : 0.0f;
+                    acc[nb][0] = fmaf(sc, cacc[nb][0], acc[nb][0]);
+                    acc[nb][1] = fmaf(sc, cacc[nb][1], acc[nb][1]);
+                }
+                // the tile ends here, or this warp's slice does
+                if (cc.sb == P.ksb - 1 || u == u_end - 1) {
+                    const bool full = tile_first_u >= u_begin && cc.sb == P.ksb - 1;
+                    tile_epilogue<NB>(acc, full, M, P.n, cc.t, P.tile_begin + cc.t, P.unit_begin + cc.t * P.ksb,
+                                      P.ksb, S, W, wid, a.partials, a.counters, a.maxc, P.y);
+#pragma unroll
+                    for (int nb = 0; nb < NB; nb++) acc[nb][0] = acc[nb][1] = 0.0f;
+                    tile_first_u = u + 1;
+                }
+                ldg_advance(a, cc);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ host side
+// Units in flight per warp and CTAs per SM.  Two CTAs (16 warps, <= 128 registers a
+// thread) with about 12 x 16 bytes in flight per lane where the registers allow it;
+// otherwise one CTA of 8 warps with twice the depth.  Either way each SM keeps about
+// 96 KB of weights in flight, twice what 1 us of HBM latency at full rate needs.
+struct LdgShape {
+    int D, CPS;
+};
+constexpr LdgShape ldg_shape(int bits, int group, int nb) {
+    const int d = bits == 2 ? 6 : bits == 3 ? 4 : bits == 4 ? 3 : 2;
+    const bool two = nb == 1 && !(group == 32 && bits >= 5);
+    if (two) return {(group == 32 && bits == 4) ? 2 : d, 2};
+    return {nb >= 4 ? d + d / 2 : 2 * d, 1};
+}
+
+struct LdgPlan {
+    int64_t total_units = 0, total_tiles = 0, total_warps = 0;
+    int grid = 1, maxc = 2;
+};
+
+static LdgPlan plan_ldg(const int64_t* n, const int64_t* k, int count, int cps) {
+    LdgPlan pl;
+    int64_t max_ksb = 1;
+    for (int i = 0; i < count; i++) {
+        const int64_t n_tiles = n[i] / 16;
+        const int64_t ksb = k[i] / kLdgChunk;
+        pl.total_units += n_tiles * ksb;
+        pl.total_tiles += n_tiles;
+        max_ksb = std::max(max_ksb, ksb);
+    }
+    pl.grid = (int)std::max<int64_t>(
+        1, std::min<int64_t>((int64_t)sm_count() * cps, ceil_div(pl.total_units, (int64_t)kLdgWarps)));
+    // no more warps than units: every participating warp then owns at least one unit,
+    // so each warp counted as a contributor to a tile also arrives at its ticket
+    pl.total_warps = std::min<int64_t>((int64_t)pl.grid * kLdgWarps, std::max<int64_t>(pl.total_units, 1));
+    // warps that share one tile: the slices are floor(w S / W), so a window of ksb units
+    // meets at most ceil(ksb W / S) + 1 of them; one more slot of margin
+    pl.maxc = (int)(ceil_div(max_ksb * pl.total_warps, std::max<int64_t>(pl.total_units, 1)) + 2);
+    return pl;
+}
+
+// Workspace: ticket header, partial tiles, then per product the planes [2M][k], the
+// group sums [M][k/32] (enough for every group size) and the exponents [M][k/256].
+static size_t al256(size_t v) { return (v + 255) / 256 * 256; }
+
+static size_t prep_bytes(int64_t k, int64_t M) {
+    return al256((size_t)(2 * M * k)) + al256((size_t)(M * (k / 32) * 4)) + al256((size_t)(M * (k / kLdgChunk) * 4));
+}
+
+// The workspace is sized for the larger grid (two CTAs per SM), which every shape fits.
+size_t gemv_group_ldg_ws_bytes_multi(const int64_t* n, const int64_t* k, int count, int64_t M) {
+    const LdgPlan pl = plan_ldg(n, k, count, 2);
+    size_t b = kCounterBytes + al256((size_t)(pl.total_tiles * pl.maxc * 16 * M * 4));
+    for (int i = 0; i < count; i++) b += prep_bytes(k[i], M);
+    return b;
+}
+
+size_t gemv_group_ldg_ws_bytes(int64_t M, int64_t n, int64_t k) { return gemv_group_ldg_ws_bytes_multi(&n, &k, 1, M); }
+
+bool gemv_group_ldg_supported(int64_t M, int64_t n, int64_t k, int bits, int group) {
+    if (M < 1 || M > 16 || k % kLdgChunk != 0 || n % 16 != 0 || bits < 2 || bits > 6) return false;
+    if (group != 32 && group != 64 && group != 128) return false;
+    if ((k / group) % 8 != 0) return false;              // 16-byte aligned scale rows
+    return n / 16 <= kMaxTiles;
+}
+
+template <class Kern, class... Args>
+static lbq_status launch_pdl(Kern kern, int grid, int threads, size_t smem, cudaStream_t st, const Args&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, args...) != cudaSuccess) return LBQ_ERR_CUDA;
+    return launch_status();
+}
+
+// Shared memory a CTA may spend on prepared activations (two CTAs per SM share 228 KB).
+static int ldg_smem_budget(int cps) { return cps == 2 ? 100 * 1024 : 200 * 1024; }
+
+template <auto KERN>
+static lbq_status ldg_smem_attr(int bytes) {
+    static bool set[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LBQ_ERR_CUDA;
+    if (dev >= 0 && dev < 64 && set[dev]) return LBQ_OK;
+    if (cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return LBQ_ERR_CUDA;
+    if (dev >= 0 && dev < 64) set[dev] = true;
+    return LBQ_OK;
+}
+
+template <int B, int GROUP, int NB>
+static lbq_status launch_ldg_inst(int grid, bool smemp, bool bf16, int smem, cudaStream_t st, const LdgArgs& args,
+                                  const PrepArgs& prep) {
+    constexpr LdgShape sh = ldg_shape(B, GROUP, NB);
+    if constexpr (NB == 1) {
+        if (smemp) {
+            constexpr auto kb = k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.CPS, true, true>;
+            constexpr auto kh = k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.CPS, true, false>;
+            const lbq_status s = bf16 ? ldg_smem_attr<kb>(ldg_smem_budget(sh.CPS))
+                                      : ldg_smem_attr<kh>(ldg_smem_budget(sh.CPS));
+            if (s != LBQ_OK) return s;
+            return launch_pdl(bf16 ? kb : kh, grid, kLdgThreads, (size_t)smem, st, args, prep);
+        }
+    }
+    return launch_pdl(k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.CPS, false, false>, grid, kLdgThreads, 0, st, args,
+                      prep);
+}
+
+template <int B, int GROUP>
+static lbq_status launch_ldg_nb(int NB, int grid, bool smemp, bool bf16, int smem, cudaStream_t st,
+                                const LdgArgs& args, const PrepArgs& prep) {
+    if (NB == 1) return launch_ldg_inst<B, GROUP, 1>(grid, smemp, bf16, smem, st, args, prep);
+    if (NB == 2) return launch_ldg_inst<B, GROUP, 2>(grid, smemp, bf16, smem, st, args, prep);
+    if (NB == 3) return launch_ldg_inst<B, GROUP, 3>(grid, smemp, bf16, smem, st, args, prep);
+    return launch_ldg_inst<B, GROUP, 4>(grid, smemp, bf16, smem, st, args, prep);
+}
+
+template <int B>
+static lbq_status launch_ldg_b(int group, int NB, int grid, bool smemp, bool bf16, int smem, cudaStream_t st,
+                               const LdgArgs& args, const PrepArgs& prep) {
+    if (group == 32) return launch_ldg_nb<B, 32>(NB, grid, smemp, bf16, smem, st, args, prep);
+    if (group == 64) return launch_ldg_nb<B, 64>(NB, grid, smemp, bf16, smem, st, args, prep);
+    return launch_ldg_nb<B, 128>(NB, grid, smemp, bf16, smem, st, args, prep);
+}
+
+static int al16(int64_t v) { return (int)((v + 15) / 16 * 16); }
+
+lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count, bool bf16, int64_t M, int bits,
+                                       int group, void* ws, size_t ws_bytes, cudaStream_t st) {
+    int64_t n[kMaxGemvProblems], k[kMaxGemvProblems];
+    for (int i = 0; i < count; i++) {
+        n[i] = probs[i].n;
+        k[i] = probs[i].k;
+    }
+    const int NB = (int)((2 * M + 7) / 8);
+    const LdgShape shape = ldg_shape(bits, group, NB);
+    const LdgPlan pl = plan_ldg(n, k, count, shape.CPS);
+    if (pl.total_units == 0) return LBQ_OK;
+    if (ws == nullptr || ws_bytes < gemv_group_ldg_ws_bytes_multi(n, k, count, M)) return LBQ_ERR_WORKSPACE;
+    if (pl.total_tiles > kMaxTiles) return LBQ_ERR_UNSUPPORTED;
+
+    LdgArgs args;
+    memset(&args, 0, sizeof args);
+    PrepArgs prep;
+    memset(&prep, 0, sizeof prep);
+    char* base = (char*)ws;
+    args.counters = (unsigned*)base;
+    args.partials = (float*)(base + kCounterBytes);
+    size_t off = kCounterBytes + al256((size_t)(pl.total_tiles * pl.maxc * 16 * M * 4));
+    int64_t ub = 0, tb = 0, pw = 0;
+    int soff = 0;
+    for (int i = 0; i < count; i++) {
+        // products that read the same activations share one prep slot
+        int slot = -1;
+        for (int j = 0; j < prep.count; j++)
+            if (prep.s[j].x == (const uint16_t*)probs[i].x && prep.s[j].k == k[i]) slot = j;
+        if (slot < 0) {
+            PrepSlot& s = prep.s[prep.count];
+            s.x = (const uint16_t*)probs[i].x;
+            s.k = k[i];
+            s.planes = (int8_t*)(base + off);
+            s.xsum = (float*)(base + off + al256((size_t)(2 * M * k[i])));
+            s.expo = (int*)(base + off + al256((size_t)(2 * M * k[i])) + al256((size_t)(M * (k[i] / 32) * 4)));
+            s.sp = soff;
+            s.sx = s.sp + al16(2 * M * k[i]);
+            s.se = s.sx + al16(M * (k[i] / group) * 4);
+            soff = s.se + al16(M * (k[i] / kLdgChunk) * 4);
+            s.warp_begin = pw;
+            pw += M * (k[i] / kLdgChunk);
+            off += prep_bytes(k[i], M);
+            slot = prep.count++;
+        }
+        LdgProblem& P = args.p[i];
+        P.packed = (const uint8_t*)probs[i].packed;
+        P.scales = (const uint16_t*)probs[i].scales;
+        P.zeros = (const uint16_t*)probs[i].zeros;
+        P.y = (uint16_t*)probs[i].y;
+        P.slot = slot;
+        P.n = n[i];
+        P.k = k[i];
+        P.ksb = k[i] / kLdgChunk;
+        P.n_tiles = n[i] / 16;
+        P.ngroups = k[i] / group;
+        P.unit_begin = ub;
+        P.tile_begin = tb;
+        ub += P.n_tiles * P.ksb;
+        tb += P.n_tiles;
+    }
+    prep.total_warps = pw;
+    prep.M = (int)M;
+    args.total_units = pl.total_units;
+    args.total_warps = pl.total_warps;
+    args.count = count;
+    args.M = (int)M;
+    args.maxc = pl.maxc;
+
+    // prepared activations in each CTA's shared memory when they fit, else one prep launch
+    const bool smemp = NB == 1 && soff <= ldg_smem_budget(shape.CPS);
+    if (!smemp) {
+        const int pgrid = (int)ceil_div(pw, (int64_t)8);
+        lbq_status s;
+#define LBQ_PREP(GR) (bf16 ? launch_pdl(k_gemv_prep<GR, true>, pgrid, 256, 0, st, prep) \
+                           : launch_pdl(k_gemv_prep<GR, false>, pgrid, 256, 0, st, prep))
+        if (group == 32) s = LBQ_PREP(32);
+        else if (group == 64) s = LBQ_PREP(64);
+        else s = LBQ_PREP(128);
+#undef LBQ_PREP
+        if (s != LBQ_OK) return s;
+    }
+    switch (bits) {
+        case 2: return launch_ldg_b<2>(group, NB, pl.grid, smemp, bf16, soff, st, args, prep);
+        case 3: return launch_ldg_b<3>(group, NB, pl.grid, smemp, bf16, soff, st, args, prep);
+        case 4: return launch_ldg_b<4>(group, NB, pl.grid, smemp, bf16, soff, st, args, prep);
+        case 5: return launch_ldg_b<5>(group, NB, pl.grid, smemp, bf16, soff, st, args, prep);
+        default: return launch_ldg_b<6>(group, NB, pl.grid, smemp, bf16, soff, st, args, prep);
+    }
+}
+
+lbq_status launch_gemv_group_ldg(const void* x, bool bf16, int64_t M, const void* packed, const void* scales,
+                                 const void* zeros, int64_t n, int64_t k, int bits, int group, void* y, void* ws,
+                                 size_t ws_bytes, cudaStream_t st) {
+    lbq_gemv_problem p;
+    p.x = x;
+    p.packed = packed;
+    p.scales = scales;
+    p.zeros = zeros;
+    p.y = y;
+    p.n = n;
+    p.k = k;
+    return launch_gemv_group_ldg_multi(&p, 1, bf16, M, bits, group, ws, ws_bytes, st);
+}
+
+}  // namespace lbq

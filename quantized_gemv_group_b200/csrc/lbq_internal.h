@@ -65,6 +65,16 @@ lbq_status launch_gemv_group_tma(const void* x, bool bf16, int64_t M, const void
                                  const void* zeros, int64_t n, int64_t k, int bits, int group, void* y, void* ws,
                                  size_t ws_bytes, cudaStream_t st);
 
+// Group GEMV with weights streamed into registers (M <= 16, kernel layout).
+bool gemv_group_ldg_supported(int64_t M, int64_t n, int64_t k, int bits, int group);
+size_t gemv_group_ldg_ws_bytes(int64_t M, int64_t n, int64_t k);
+size_t gemv_group_ldg_ws_bytes_multi(const int64_t* n, const int64_t* k, int count, int64_t M);
+lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count, bool bf16, int64_t M, int bits,
+                                       int group, void* ws, size_t ws_bytes, cudaStream_t st);
+lbq_status launch_gemv_group_ldg(const void* x, bool bf16, int64_t M, const void* packed, const void* scales,
+                                 const void* zeros, int64_t n, int64_t k, int bits, int group, void* y, void* ws,
+                                 size_t ws_bytes, cudaStream_t st);
+
 // Batched group GEMM on tcgen05 (M >= 64, kernel layout).
 size_t gemm_group_tc_ws_bytes(int64_t M, int64_t n, int64_t k);
 bool gemm_group_tc_supported(int64_t M, int64_t n, int64_t k, int bits, int group);

@@ -57,10 +57,10 @@ extern "C" lbq_status lbq_gemv_group_noalloc(const void* x, lbq_dtype x_dtype, i
         return LBQ_ERR_INVALID_ARG;
     if (M == 0 || n == 0) return LBQ_OK;
     if (!x || !packed || !scales || !zeros || !y) return LBQ_ERR_INVALID_ARG;
-    if (!gemv_group_tma_supported(M, n, k, bits, group)) return LBQ_ERR_UNSUPPORTED;
+    if (!gemv_group_ldg_supported(M, n, k, bits, group)) return LBQ_ERR_UNSUPPORTED;
     const uintptr_t al = (uintptr_t)x | (uintptr_t)packed | (uintptr_t)scales | (uintptr_t)zeros;
     if ((al % 16) != 0 || ((uintptr_t)y % 2) != 0) return LBQ_ERR_MISALIGNED;
-    const size_t need = gemv_group_tma_ws_bytes(M, n, k);
+    const size_t need = gemv_group_ldg_ws_bytes(M, n, k);
     if (need > kScratchBytes) return LBQ_ERR_SCRATCH_LIMIT;
     void* ws = scratch_address();
     if (!ws) return LBQ_ERR_CUDA;
@@ -68,6 +68,6 @@ extern "C" lbq_status lbq_gemv_group_noalloc(const void* x, lbq_dtype x_dtype, i
     // them zero, but the array keeps whatever the previous call left, so clear them.
     const size_t used_counters = (size_t)(n / 16) * sizeof(unsigned);
     if (cudaMemsetAsync(ws, 0, used_counters, (cudaStream_t)stream) != cudaSuccess) return LBQ_ERR_CUDA;
-    return launch_gemv_group_tma(x, x_dtype == LBQ_BF16, M, packed, scales, zeros, n, k, bits, group, y, ws,
+    return launch_gemv_group_ldg(x, x_dtype == LBQ_BF16, M, packed, scales, zeros, n, k, bits, group, y, ws,
                                  kScratchBytes, (cudaStream_t)stream);
 }
