@@ -60,7 +60,14 @@ struct LdgArgs {
     unsigned* counters;
     int64_t total_units, total_warps;
     int count, M, maxc;
+    int sring;              // byte offset of the scale/zero rings in shared memory
+    int szero;              // byte offset of a 256-byte zero chunk in shared memory
 };
+
+constexpr int kScaleRing = 6;               // units of scales/zeros in flight per warp
+
+// Bytes of one unit's scale/zero slot: 2 arrays x 16 rows x (256 / GROUP) fp16.
+constexpr int scale_slot_bytes(int group) { return 64 * (kLdgChunk / group); }
 
 // Prepared activations of one distinct x: planes [2M][k] (row 2m = hi plane of token m,
 // 2m + 1 = lo plane, B-fragment byte order), exact group sums [M][k / GROUP] and
@@ -77,6 +84,7 @@ struct PrepSlot {
 
 struct PrepArgs {
     PrepSlot s[kMaxGemvProblems];
+    int8_t* zero;           // 256 zero bytes in global memory (written by k_gemv_prep)
     int64_t total_warps;
     int count, M;
 };
@@ -111,21 +119,22 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p, uint64_t pol) {
     return v;
 }
 
-// NG consecutive fp16 values (NG in 2, 4, 8; 2 * NG-byte aligned) through L1.
+// NG consecutive fp16 values (NG in 4, 8, 16; 2 * NG-byte aligned) from shared memory.
 template <int NG>
-__device__ __forceinline__ void ldg_halves(const uint16_t* p, uint32_t (&d)[NG / 2]) {
-    if constexpr (NG == 2) {
-        d[0] = __ldg(reinterpret_cast<const unsigned int*>(p));
-    } else if constexpr (NG == 4) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+__device__ __forceinline__ void lds_halves_ldg(const uint16_t* p, uint32_t (&d)[NG / 2]) {
+    if constexpr (NG == 4) {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
         d[0] = v.x;
         d[1] = v.y;
     } else {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-        d[0] = v.x;
-        d[1] = v.y;
-        d[2] = v.z;
-        d[3] = v.w;
+#pragma unroll
+        for (int i = 0; i < NG / 8; i++) {
+            const uint4 v = reinterpret_cast<const uint4*>(p)[i];
+            d[4 * i] = v.x;
+            d[4 * i + 1] = v.y;
+            d[4 * i + 2] = v.z;
+            d[4 * i + 3] = v.w;
+        }
     }
 }
 
@@ -135,15 +144,23 @@ __device__ __forceinline__ void ldg_halves(const uint16_t* p, uint32_t (&d)[NG /
 // 4(l mod 4).. (even elements) and 16 + 4(l mod 4).. (odd elements) of k-step l / 4.
 // x may have been written by the previous kernel of the stream, so it is read through
 // L2 (ld.global.cg), never through the non-coherent path.
+// Byte offset, inside a 256-wide chunk of a plane row, of the 8 bytes prepared by lane l
+// (elements 8l..8l+7): k-step l / 4, lane-group l mod 4; two consecutive k-steps of a
+// lane-group sit side by side so that one 16-byte load fetches both B fragments.
+__host__ __device__ __forceinline__ int plane_off(int l) { return 64 * (l >> 3) + 16 * (l & 3) + 8 * ((l >> 2) & 1); }
+
 struct PrepOut {
     uint2 hi, lo;   // this lane's 8 bytes of the hi and lo planes
     int gsum;       // exact sum of v over the lane's group (valid on the group's first lane)
     int E;
 };
 
+__device__ __forceinline__ uint4 prep_load(const uint16_t* xc, int lane) {
+    return __ldcg(reinterpret_cast<const uint4*>(xc + 8 * lane));
+}
+
 template <int GROUP, bool BF16>
-__device__ __forceinline__ PrepOut prep_chunk(const uint16_t* xc, int lane) {
-    const uint4 raw = __ldcg(reinterpret_cast<const uint4*>(xc + 8 * lane));
+__device__ __forceinline__ PrepOut prep_convert(const uint4 raw) {
     const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
     float v[8];
     float mx = 0.0f;
@@ -185,6 +202,11 @@ __device__ __forceinline__ PrepOut prep_chunk(const uint16_t* xc, int lane) {
     return r;
 }
 
+template <int GROUP, bool BF16>
+__device__ __forceinline__ PrepOut prep_chunk(const uint16_t* xc, int lane) {
+    return prep_convert<GROUP, BF16>(prep_load(xc, lane));
+}
+
 // Warp task wi of the prep list -> (slot, token, chunk).
 __device__ __forceinline__ int prep_task(const PrepArgs& a, int64_t wi, int& m, int64_t& ch) {
     int s = 0;
@@ -209,8 +231,9 @@ __global__ void __launch_bounds__(256) k_gemv_prep(const __grid_constant__ PrepA
     const PrepSlot& S = a.s[prep_task(a, wi, m, ch)];
     const PrepOut r = prep_chunk<GROUP, BF16>(S.x + (int64_t)m * S.k + ch * kLdgChunk, lane);
     int8_t* row_h = S.planes + (int64_t)(2 * m) * S.k + ch * kLdgChunk;
-    *reinterpret_cast<uint2*>(row_h + 8 * lane) = r.hi;
-    *reinterpret_cast<uint2*>(row_h + S.k + 8 * lane) = r.lo;
+    *reinterpret_cast<uint2*>(row_h + plane_off(lane)) = r.hi;
+    *reinterpret_cast<uint2*>(row_h + S.k + plane_off(lane)) = r.lo;
+    if (wi == 0 && lane < 16) reinterpret_cast<uint4*>(a.zero)[lane] = make_uint4(0, 0, 0, 0);
     constexpr int LPG = GROUP / 8;
     if (lane % LPG == 0) S.xsum[(int64_t)m * (S.k / GROUP) + ch * (kLdgChunk / GROUP) + lane / LPG] = (float)r.gsum;
     if (lane == 0) S.expo[(int64_t)m * (S.k / kLdgChunk) + ch] = r.E;
@@ -219,9 +242,27 @@ __global__ void __launch_bounds__(256) k_gemv_prep(const __grid_constant__ PrepA
 // Prepared-activation reads: shared memory (plain loads) or global memory written by the
 // prep kernel of this launch (L2 only: data another grid wrote during this grid's life).
 template <bool SMEMP>
-__device__ __forceinline__ uint2 ld_plane(const int8_t* p) {
-    if constexpr (SMEMP) return *reinterpret_cast<const uint2*>(p);
-    else return __ldcg(reinterpret_cast<const uint2*>(p));
+__device__ __forceinline__ uint4 ld_plane16(const int8_t* p) {
+    if constexpr (SMEMP) return *reinterpret_cast<const uint4*>(p);
+    else return __ldcg(reinterpret_cast<const uint4*>(p));
+}
+template <bool SMEMP, int N>
+__device__ __forceinline__ void ld_floats(const float* p, float (&v)[N]) {
+    if constexpr (N == 2) {
+        const float2 t = SMEMP ? *reinterpret_cast<const float2*>(p) : __ldcg(reinterpret_cast<const float2*>(p));
+        v[0] = t.x;
+        v[1] = t.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; i += 4) {
+            const float4 t =
+                SMEMP ? *reinterpret_cast<const float4*>(p + i) : __ldcg(reinterpret_cast<const float4*>(p + i));
+            v[i] = t.x;
+            v[i + 1] = t.y;
+            v[i + 2] = t.z;
+            v[i + 3] = t.w;
+        }
+    }
 }
 template <bool SMEMP, class T>
 __device__ __forceinline__ T ld_prep(const T* p) {
@@ -230,21 +271,6 @@ __device__ __forceinline__ T ld_prep(const T* p) {
 }
 
 // ------------------------------------------------------------------ GEMV
-struct LdgCursor {
-    int p;
-    int64_t t, sb;
-};
-
-__device__ __forceinline__ void ldg_advance(const LdgArgs& a, LdgCursor& cu) {
-    if (++cu.sb == a.p[cu.p].ksb) {
-        cu.sb = 0;
-        if (++cu.t == a.p[cu.p].n_tiles) {
-            cu.t = 0;
-            if (cu.p + 1 < a.count) cu.p++;
-        }
-    }
-}
-
 // D units in flight per warp; CPS resident CTAs per SM (2: up to 128 registers a thread);
 // SMEMP: every CTA prepares the activations itself, in its shared memory, right after
 // waiting for the previous kernel (else they come from k_gemv_prep via L2).
@@ -263,44 +289,80 @@ __global__ void __launch_bounds__(kLdgThreads, CPS)
     const int g = lane >> 2, c = lane & 3;
     const int64_t W = a.total_warps, S = a.total_units;
     const int64_t wid = (int64_t)blockIdx.x * kLdgWarps + warp;
-    // warps past the W that share the list (grid * 8 may exceed it) take no units
-    const int64_t u_begin = wid < W ? wid * S / W : S;
-    const int64_t u_end = wid < W ? (wid + 1) * S / W : S;
+    // warps past the W that share the list (grid * 8 may exceed it) take no units;
+    // unit indices fit 32 bits (the host caps the list)
+    const int u_begin = (int)(wid < W ? wid * S / W : S);
+    const int u_end = (int)(wid < W ? (wid + 1) * S / W : S);
     const int M = a.M;
     const uint64_t pol = l2_policy_evict_first();
 
     const bool has_work = u_begin < u_end;
-    LdgCursor cc;
-    cc.p = 0;
-    while (cc.p + 1 < a.count && u_begin >= a.p[cc.p + 1].unit_begin) cc.p++;
+    const int arr = lane >> 4, srow = lane & 15;     // this lane's row of the scale ring fill
+
+    // compute cursor (problem cp, tile ct, superblock csb), weight-load cursor (pointer,
+    // units left in its problem) and scale-fill cursor (row pointer, tile, superblock)
+    int cp = 0;
+    while (cp + 1 < a.count && u_begin >= a.p[cp + 1].unit_begin) cp++;
+    int ct = 0, csb = 0;
     if (has_work) {
-        const int64_t lu = u_begin - a.p[cc.p].unit_begin;
-        cc.t = lu / a.p[cc.p].ksb;
-        cc.sb = lu % a.p[cc.p].ksb;
+        const int lu = u_begin - (int)a.p[cp].unit_begin;
+        ct = lu / (int)a.p[cp].ksb;
+        csb = lu % (int)a.p[cp].ksb;
     }
-    LdgCursor lc = cc;
+    int lp = cp;
+    const uint8_t* lptr = a.p[cp].packed + ((int64_t)ct * a.p[cp].ksb + csb) * (512 * B) + 16 * lane;
+    int lleft = (int)(a.p[cp].n_tiles * a.p[cp].ksb) - (ct * (int)a.p[cp].ksb + csb);
+    int sp = cp;
+    int st_ = ct, ssb = csb;
+    const uint16_t* sbase = (arr ? a.p[cp].zeros : a.p[cp].scales) + ((int64_t)ct * 16 + srow) * a.p[cp].ngroups;
 
     uint4 wb[D][B];
-    auto load_unit = [&](uint4 (&dst)[B], const LdgCursor& cu) {
-        const LdgProblem& P = a.p[cu.p];
-        const uint8_t* src = P.packed + (cu.t * P.ksb + cu.sb) * (int64_t)(512 * B) + 16 * lane;
+    auto load_next = [&](uint4 (&dst)[B]) {
 #pragma unroll
-        for (int i = 0; i < B; i++) dst[i] = ldg_stream(src + 512 * i, pol);
+        for (int i = 0; i < B; i++) dst[i] = ldg_stream(lptr + 512 * i, pol);
+        lptr += 512 * B;
+        if (--lleft == 0 && lp + 1 < a.count) {
+            lp++;
+            lptr = a.p[lp].packed + 16 * lane;
+            lleft = (int)(a.p[lp].n_tiles * a.p[lp].ksb);
+        }
     };
+    // scale/zero ring: lane i copies, for one unit, row i mod 16 of the scales (i < 16)
+    // or of the zeros into the warp's slot, rows interleaved [row][scales, zeros]
+    constexpr int SCB = scale_slot_bytes(GROUP);
+    uint8_t* sring = smem + a.sring + warp * kScaleRing * SCB;
+    auto issue_scales = [&](int slot) {
+        cp_async_ca<2 * NGC>(smem_u32(sring + slot * SCB + (srow * 2 + arr) * 2 * NGC), sbase + ssb * NGC);
+        if (++ssb == a.p[sp].ksb) {
+            ssb = 0;
+            if (++st_ == a.p[sp].n_tiles && sp + 1 < a.count) {
+                sp++;
+                st_ = 0;
+                sbase = (arr ? a.p[sp].zeros : a.p[sp].scales) + srow * a.p[sp].ngroups;
+            } else {
+                sbase += 16 * a.p[sp].ngroups;
+            }
+        }
+    };
+#pragma unroll 1
+    for (int i = 0; i < kScaleRing; i++) {
+        if (u_begin + i < u_end) issue_scales(i);
+        cp_async_commit();
+    }
     // prologue: the first D units' weights (into registers) and the next PF (into L2)
     // do not depend on the previous kernels
 #pragma unroll
-    for (int d = 0; d < D; d++) {
-        if (u_begin + d < u_end) {
-            load_unit(wb[d], lc);
-            ldg_advance(a, lc);
-        }
-    }
-    if (lane < PF && u_begin + D + lane < u_end) {
-        LdgCursor pc = lc;
-        for (int i = 0; i < lane; i++) ldg_advance(a, pc);
-        const LdgProblem& P = a.p[pc.p];
-        l2_prefetch_bulk(P.packed + (pc.t * P.ksb + pc.sb) * (int64_t)(512 * B), 512 * B);
+    for (int d = 0; d < D; d++)
+        if (u_begin + d < u_end) load_next(wb[d]);
+    if (lane < PF && u_begin + D + lane < u_end && lleft > lane)
+        l2_prefetch_bulk(lptr - 16 * lane + (int64_t)lane * (512 * B), 512 * B);
+    // zeroed chunk that padded plane rows and tokens read instead of branching
+    const int8_t* zero;
+    if constexpr (SMEMP) {
+        if (threadIdx.x < 16) reinterpret_cast<uint4*>(smem + a.szero)[threadIdx.x] = make_uint4(0, 0, 0, 0);
+        zero = reinterpret_cast<const int8_t*>(smem + a.szero);
+    } else {
+        zero = pa.zero;
     }
     griddep_wait();
     if constexpr (SMEMP) {
@@ -311,29 +373,57 @@ __global__ void __launch_bounds__(kLdgThreads, CPS)
             const PrepSlot& Q = pa.s[prep_task(pa, wi, m, ch)];
             const PrepOut r = prep_chunk<GROUP, BF16>(Q.x + (int64_t)m * Q.k + ch * kLdgChunk, lane);
             int8_t* row_h = reinterpret_cast<int8_t*>(smem + Q.sp) + (int64_t)(2 * m) * Q.k + ch * kLdgChunk;
-            *reinterpret_cast<uint2*>(row_h + 8 * lane) = r.hi;
-            *reinterpret_cast<uint2*>(row_h + Q.k + 8 * lane) = r.lo;
+            *reinterpret_cast<uint2*>(row_h + plane_off(lane)) = r.hi;
+            *reinterpret_cast<uint2*>(row_h + Q.k + plane_off(lane)) = r.lo;
             constexpr int LPG = GROUP / 8;
             if (lane % LPG == 0)
                 reinterpret_cast<float*>(smem + Q.sx)[(int64_t)m * (Q.k / GROUP) + ch * (kLdgChunk / GROUP) +
                                                       lane / LPG] = (float)r.gsum;
             if (lane == 0) reinterpret_cast<int*>(smem + Q.se)[(int64_t)m * (Q.k / kLdgChunk) + ch] = r.E;
         }
-        __syncthreads();
     }
+    __syncthreads();
     if (!has_work) return;
+
+    // per-problem byte offsets, from one base, of this lane's plane rows, group sums and
+    // exponents; padded rows and tokens point at the zero chunk with a zero stride
+    const char* pbase = nullptr;
+    int prow0[NB], xrow0[NB], erow0[NB], pstep[NB], xstep[NB];
+    auto set_problem_bases = [&]() {
+        const LdgProblem& P = a.p[cp];
+        const PrepSlot& PS = pa.s[P.slot];
+        const char* planes = SMEMP ? reinterpret_cast<const char*>(smem + PS.sp) : reinterpret_cast<const char*>(PS.planes);
+        const char* xsum = SMEMP ? reinterpret_cast<const char*>(smem + PS.sx) : reinterpret_cast<const char*>(PS.xsum);
+        const char* expo = SMEMP ? reinterpret_cast<const char*>(smem + PS.se) : reinterpret_cast<const char*>(PS.expo);
+        pbase = planes;
+        const int zoff = (int)(reinterpret_cast<const char*>(zero) - planes);
+        const int xoff = (int)(xsum - planes), eoff = (int)(expo - planes);
+#pragma unroll
+        for (int nb = 0; nb < NB; nb++) {
+            const int pl = 8 * nb + g;
+            const bool pv = pl < 2 * M;
+            prow0[nb] = pv ? pl * (int)P.k + 16 * c : zoff + 16 * c;
+            pstep[nb] = pv ? kLdgChunk : 0;
+            const int tok = 4 * nb + c;
+            const bool tv = tok < M;
+            xrow0[nb] = tv ? xoff + 4 * tok * (int)P.ngroups : zoff;
+            erow0[nb] = tv ? eoff + 4 * tok * (int)P.ksb : zoff;
+            xstep[nb] = tv ? 4 : 0;
+        }
+    };
+    set_problem_bases();
 
     float acc[NB][2];
 #pragma unroll
     for (int nb = 0; nb < NB; nb++) acc[nb][0] = acc[nb][1] = 0.0f;
-    int64_t tile_first_u = u_begin - cc.sb;        // first unit of the tile being accumulated
+    int tile_first_u = u_begin - csb;              // first unit of the tile being accumulated
+    int rs = 0;                                    // ring slot of the unit being computed
 
-    for (int64_t base = u_begin; base < u_end; base += D) {
+    for (int base = u_begin; base < u_end; base += D) {
 #pragma unroll
         for (int d = 0; d < D; d++) {
-            const int64_t u = base + d;
+            const int u = base + d;
             if (u < u_end) {
-                const LdgProblem& P = a.p[cc.p];
                 uint32_t lo[F::NLO], hi[F::NHI];
 #pragma unroll
                 for (int i = 0; i < G::W0; i++) {
@@ -350,37 +440,25 @@ __global__ void __launch_bounds__(kLdgThreads, CPS)
                     hi[4 * i + 3] = wb[d][G::W0 + i].w;
                 }
                 if constexpr (G::W1 == 0) hi[0] = 0;
-                // refill this slot with the unit D ahead
-                if (u + D < u_end) {
-                    load_unit(wb[d], lc);
-                    ldg_advance(a, lc);
-                }
-                // scales and zeros of this unit's NGC groups, rows g and g+8
-                const int64_t rl = cc.t * 16 + g;
-                const int64_t j0 = cc.sb * NGC;
-                uint32_t sh0[NGC / 2], sh1[NGC / 2], zh0[NGC / 2], zh1[NGC / 2];
-                ldg_halves<NGC>(P.scales + rl * P.ngroups + j0, sh0);
-                ldg_halves<NGC>(P.scales + (rl + 8) * P.ngroups + j0, sh1);
-                ldg_halves<NGC>(P.zeros + rl * P.ngroups + j0, zh0);
-                ldg_halves<NGC>(P.zeros + (rl + 8) * P.ngroups + j0, zh1);
-                // prepared activations of this product's x
-                const PrepSlot& PS = pa.s[P.slot];
-                const int8_t* planes = SMEMP ? reinterpret_cast<const int8_t*>(smem + PS.sp) : PS.planes;
-                const float* xsum = SMEMP ? reinterpret_cast<const float*>(smem + PS.sx) : PS.xsum;
-                const int* expo = SMEMP ? reinterpret_cast<const int*>(smem + PS.se) : PS.expo;
-                // B-fragment rows: plane 8*nb + g (token (8*nb + g)/2, hi or lo)
-                const int8_t* prow[NB];
-                bool pval[NB];
+                // refill this register slot with the unit D ahead
+                if (u + D < u_end) load_next(wb[d]);
+                // scales and zeros of this unit's NGC groups, rows g and g+8, from the ring
+                cp_async_wait<kScaleRing - 1>();
+                __syncwarp();
+                const uint16_t* sslot = reinterpret_cast<const uint16_t*>(sring + rs * SCB);
+                uint32_t sz0[NGC], sz1[NGC];        // [scales NGC/2 words | zeros NGC/2 words]
+                lds_halves_ldg<2 * NGC>(sslot + (2 * g) * NGC, sz0);
+                lds_halves_ldg<2 * NGC>(sslot + (2 * (g + 8)) * NGC, sz1);
+                // exponent of each token of this lane, this unit
+                int E[NB];
 #pragma unroll
-                for (int nb = 0; nb < NB; nb++) {
-                    const int pl = 8 * nb + g;
-                    pval[nb] = pl < 2 * M;
-                    prow[nb] = planes + (int64_t)(pval[nb] ? pl : 0) * P.k + cc.sb * kLdgChunk + 8 * c;
-                }
+                for (int nb = 0; nb < NB; nb++)
+                    E[nb] = ld_prep<SMEMP>(reinterpret_cast<const int*>(pbase + erow0[nb] + csb * xstep[nb]));
                 float cacc[NB][2];
 #pragma unroll
                 for (int nb = 0; nb < NB; nb++) cacc[nb][0] = cacc[nb][1] = 0.0f;
                 int ci[NB][4];
+                uint4 bq[NB];
                 static_for<0, 8>([&](auto kap_c) {
                     constexpr int kap = decltype(kap_c)::value;
                     const uint32_t a0 = F::template reg<kap, 0, 0>(lo, hi);
@@ -389,21 +467,26 @@ __global__ void __launch_bounds__(kLdgThreads, CPS)
                     const uint32_t a3 = F::template reg<kap, 1, 1>(lo, hi);
 #pragma unroll
                     for (int nb = 0; nb < NB; nb++) {
-                        uint2 bv = make_uint2(0u, 0u);
-                        if (pval[nb]) bv = ld_plane<SMEMP>(prow[nb] + 32 * kap);
-                        if constexpr (kap % KPG == 0) mma_16832_u8s8_zc(ci[nb], a0, a1, a2, a3, bv.x, bv.y);
-                        else mma_16832_u8s8(ci[nb], a0, a1, a2, a3, bv.x, bv.y);
+                        // one 16-byte load holds the B fragments of k-steps kap and kap + 1
+                        if constexpr (kap % 2 == 0)
+                            bq[nb] = ld_plane16<SMEMP>(reinterpret_cast<const int8_t*>(pbase + prow0[nb] + csb * pstep[nb] +
+                                                                                        64 * (kap / 2)));
+                        const uint32_t b0 = kap % 2 ? bq[nb].z : bq[nb].x;
+                        const uint32_t b1 = kap % 2 ? bq[nb].w : bq[nb].y;
+                        if constexpr (kap % KPG == 0) mma_16832_u8s8_zc(ci[nb], a0, a1, a2, a3, b0, b1);
+                        else mma_16832_u8s8(ci[nb], a0, a1, a2, a3, b0, b1);
                     }
                     if constexpr (kap % KPG == KPG - 1) {
                         constexpr int gi = kap / KPG;
-                        const float sg = __half2float(__ushort_as_half((uint16_t)(sh0[gi / 2] >> (16 * (gi & 1)))));
-                        const float sg8 = __half2float(__ushort_as_half((uint16_t)(sh1[gi / 2] >> (16 * (gi & 1)))));
-                        const float zg = __half2float(__ushort_as_half((uint16_t)(zh0[gi / 2] >> (16 * (gi & 1)))));
-                        const float zg8 = __half2float(__ushort_as_half((uint16_t)(zh1[gi / 2] >> (16 * (gi & 1)))));
+                        constexpr int wz = NGC / 2 + gi / 2, ws = gi / 2, sh = 16 * (gi & 1);
+                        const float sg = __half2float(__ushort_as_half((uint16_t)(sz0[ws] >> sh)));
+                        const float sg8 = __half2float(__ushort_as_half((uint16_t)(sz1[ws] >> sh)));
+                        const float zg = __half2float(__ushort_as_half((uint16_t)(sz0[wz] >> sh)));
+                        const float zg8 = __half2float(__ushort_as_half((uint16_t)(sz1[wz] >> sh)));
 #pragma unroll
                         for (int nb = 0; nb < NB; nb++) {
-                            const int tok = 4 * nb + c;
-                            const float X = tok < M ? ld_prep<SMEMP>(xsum + tok * P.ngroups + j0 + gi) : 0.0f;
+                            const float X = ld_prep<SMEMP>(
+                                reinterpret_cast<const float*>(pbase + xrow0[nb] + (csb * NGC + gi) * xstep[nb]));
                             const float f0 = fmaf(-zg, X, (float)(256 * ci[nb][0] + ci[nb][1]));
                             const float f1 = fmaf(-zg8, X, (float)(256 * ci[nb][2] + ci[nb][3]));
                             cacc[nb][0] = fmaf(sg, f0, cacc[nb][0]);
@@ -411,23 +494,35 @@ __global__ void __launch_bounds__(kLdgThreads, CPS)
                         }
                     }
                 });
+                // the ring slot's values are consumed: refill it with the unit kScaleRing ahead
+                __syncwarp();
+                if (u + kScaleRing < u_end) issue_scales(rs);
+                cp_async_commit();
+                rs = rs + 1 == kScaleRing ? 0 : rs + 1;
 #pragma unroll
                 for (int nb = 0; nb < NB; nb++) {
-                    const int tok = 4 * nb + c;
-                    const float sc = tok < M ? ldg_exp2i(ld_prep<SMEMP>(expo + tok * P.ksb + cc.sb)) : 0.0f;
+                    const float sc = ldg_exp2i(E[nb]);
                     acc[nb][0] = fmaf(sc, cacc[nb][0], acc[nb][0]);
                     acc[nb][1] = fmaf(sc, cacc[nb][1], acc[nb][1]);
                 }
                 // the tile ends here, or this warp's slice does
-                if (cc.sb == P.ksb - 1 || u == u_end - 1) {
-                    const bool full = tile_first_u >= u_begin && cc.sb == P.ksb - 1;
-                    tile_epilogue<NB>(acc, full, M, P.n, cc.t, P.tile_begin + cc.t, P.unit_begin + cc.t * P.ksb,
-                                      P.ksb, S, W, wid, a.partials, a.counters, a.maxc, P.y);
+                const LdgProblem& P = a.p[cp];
+                if (csb == P.ksb - 1 || u == u_end - 1) {
+                    const bool full = tile_first_u >= u_begin && csb == P.ksb - 1;
+                    tile_epilogue<NB>(acc, full, M, P.n, ct, P.tile_begin + ct, P.unit_begin + ct * P.ksb, P.ksb, S, W,
+                                      wid, a.partials, a.counters, a.maxc, P.y);
 #pragma unroll
                     for (int nb = 0; nb < NB; nb++) acc[nb][0] = acc[nb][1] = 0.0f;
                     tile_first_u = u + 1;
                 }
-                ldg_advance(a, cc);
+                if (++csb == P.ksb) {
+                    csb = 0;
+                    if (++ct == P.n_tiles && cp + 1 < a.count) {
+                        cp++;
+                        ct = 0;
+                        set_problem_bases();
+                    }
+                }
             }
         }
     }
@@ -442,7 +537,7 @@ struct LdgShape {
     int D, CPS;
 };
 constexpr LdgShape ldg_shape(int bits, int group, int nb) {
-    const int d = bits == 2 ? 6 : bits == 3 ? 4 : bits == 4 ? 3 : 2;
+    const int d = bits == 2 ? 5 : bits == 3 ? 3 : bits == 4 ? 3 : 2;
     const bool two = nb == 1 && !(group == 32 && bits >= 5);
     if (two) return {(group == 32 && bits == 4) ? 2 : d, 2};
     return {nb >= 4 ? d + d / 2 : 2 * d, 1};
@@ -487,7 +582,7 @@ size_t gemv_group_ldg_ws_bytes_multi(const int64_t* n, const int64_t* k, int cou
     const LdgPlan pl = plan_ldg(n, k, count, 2);
     size_t b = kCounterBytes + al256((size_t)(pl.total_tiles * pl.maxc * 16 * M * 4));
     for (int i = 0; i < count; i++) b += prep_bytes(k[i], M);
-    return b;
+    return b + 256;                                      // zero chunk
 }
 
 size_t gemv_group_ldg_ws_bytes(int64_t M, int64_t n, int64_t k) { return gemv_group_ldg_ws_bytes_multi(&n, &k, 1, M); }
@@ -496,7 +591,8 @@ bool gemv_group_ldg_supported(int64_t M, int64_t n, int64_t k, int bits, int gro
     if (M < 1 || M > 16 || k % kLdgChunk != 0 || n % 16 != 0 || bits < 2 || bits > 6) return false;
     if (group != 32 && group != 64 && group != 128) return false;
     if ((k / group) % 8 != 0) return false;              // 16-byte aligned scale rows
-    return n / 16 <= kMaxTiles;
+    // 32-bit unit indices and prepared-activation offsets inside the kernel
+    return n / 16 <= kMaxTiles && k <= ((int64_t)1 << 22);
 }
 
 template <class Kern, class... Args>
@@ -544,8 +640,8 @@ static lbq_status launch_ldg_inst(int grid, bool smemp, bool bf16, int smem, cud
             return launch_pdl(bf16 ? kb : kh, grid, kLdgThreads, (size_t)smem, st, args, prep);
         }
     }
-    return launch_pdl(k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.CPS, false, false>, grid, kLdgThreads, 0, st, args,
-                      prep);
+    return launch_pdl(k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.CPS, false, false>, grid, kLdgThreads, (size_t)smem,
+                      st, args, prep);
 }
 
 template <int B, int GROUP>
@@ -579,7 +675,7 @@ lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count,
     const LdgPlan pl = plan_ldg(n, k, count, shape.CPS);
     if (pl.total_units == 0) return LBQ_OK;
     if (ws == nullptr || ws_bytes < gemv_group_ldg_ws_bytes_multi(n, k, count, M)) return LBQ_ERR_WORKSPACE;
-    if (pl.total_tiles > kMaxTiles) return LBQ_ERR_UNSUPPORTED;
+    if (pl.total_tiles > kMaxTiles || pl.total_units >= ((int64_t)1 << 31)) return LBQ_ERR_UNSUPPORTED;
 
     LdgArgs args;
     memset(&args, 0, sizeof args);
@@ -628,6 +724,7 @@ lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count,
         ub += P.n_tiles * P.ksb;
         tb += P.n_tiles;
     }
+    prep.zero = (int8_t*)(base + off);                   // 256 zero bytes after the prep slots
     prep.total_warps = pw;
     prep.M = (int)M;
     args.total_units = pl.total_units;
@@ -636,8 +733,13 @@ lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count,
     args.M = (int)M;
     args.maxc = pl.maxc;
 
-    // prepared activations in each CTA's shared memory when they fit, else one prep launch
-    const bool smemp = NB == 1 && soff <= ldg_smem_budget(shape.CPS);
+    // prepared activations in each CTA's shared memory when they fit, else one prep launch;
+    // the scale/zero rings follow them (or start the shared memory)
+    const int ring = kLdgWarps * kScaleRing * scale_slot_bytes(group);
+    const bool smemp = NB == 1 && soff + ring + 256 <= ldg_smem_budget(shape.CPS);
+    args.sring = smemp ? al16(soff) : 0;
+    args.szero = args.sring + ring;
+    const int smem = args.szero + 256;
     if (!smemp) {
         const int pgrid = (int)ceil_div(pw, (int64_t)8);
         lbq_status s;
@@ -650,11 +752,11 @@ lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count,
         if (s != LBQ_OK) return s;
     }
     switch (bits) {
-        case 2: return launch_ldg_b<2>(group, NB, pl.grid, smemp, bf16, soff, st, args, prep);
-        case 3: return launch_ldg_b<3>(group, NB, pl.grid, smemp, bf16, soff, st, args, prep);
-        case 4: return launch_ldg_b<4>(group, NB, pl.grid, smemp, bf16, soff, st, args, prep);
-        case 5: return launch_ldg_b<5>(group, NB, pl.grid, smemp, bf16, soff, st, args, prep);
-        default: return launch_ldg_b<6>(group, NB, pl.grid, smemp, bf16, soff, st, args, prep);
+        case 2: return launch_ldg_b<2>(group, NB, pl.grid, smemp, bf16, smem, st, args, prep);
+        case 3: return launch_ldg_b<3>(group, NB, pl.grid, smemp, bf16, smem, st, args, prep);
+        case 4: return launch_ldg_b<4>(group, NB, pl.grid, smemp, bf16, smem, st, args, prep);
+        case 5: return launch_ldg_b<5>(group, NB, pl.grid, smemp, bf16, smem, st, args, prep);
+        default: return launch_ldg_b<6>(group, NB, pl.grid, smemp, bf16, smem, st, args, prep);
     }
 }
 
