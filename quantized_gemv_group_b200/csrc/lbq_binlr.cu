@@ -61,7 +61,10 @@ static BinWs bin_ws(void* base, int64_t M, int64_t d_out, int64_t d_in, int64_t 
 }
 
 size_t gemv_binlr_ws_bytes(int64_t M, int64_t d_out, int64_t d_in, int64_t r, lbq_layout layout) {
-    return bin_ws(nullptr, M, d_out, d_in, r, layout).bytes;
+    size_t b = bin_ws(nullptr, M, d_out, d_in, r, layout).bytes;
+    if (layout == LBQ_LAYOUT_KERNEL && gemv_binlr_ldg_supported(M, d_out, d_in, r))
+        b = std::max(b, gemv_binlr_ldg_ws_bytes(M, d_out, d_in, r));
+    return b;
 }
 
 // ------------------------------------------------------------------ fixed-point planes
@@ -348,6 +351,11 @@ lbq_status launch_gemv_binlr(const void* x, bool bf16, int64_t M, const void* U,
                              const void* s2, int64_t d_out, int64_t d_in, int64_t r, lbq_layout layout, void* y,
                              void* ws, size_t ws_bytes, cudaStream_t st) {
     if (M == 0 || d_out == 0) return LBQ_OK;
+    // few tokens: the two-launch register-streaming path (lbq_binlr_ldg.cu)
+    // (16-byte vector loads of x and s2)
+    if (layout == LBQ_LAYOUT_KERNEL && gemv_binlr_ldg_supported(M, d_out, d_in, r) &&
+        ((uintptr_t)x | (uintptr_t)s2) % 16 == 0)
+        return launch_gemv_binlr_ldg(x, bf16, M, U, Vt, s1, s2, d_out, d_in, r, y, ws, ws_bytes, st);
     const BinWs w = bin_ws(ws, M, d_out, d_in, r, layout);
     if (ws == nullptr || ws_bytes < w.bytes) return LBQ_ERR_WORKSPACE;
     auto* xp = (const uint16_t*)x;

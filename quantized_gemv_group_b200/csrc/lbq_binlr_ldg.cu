@@ -1,0 +1,365 @@
+// lbq_binlr_ldg.cu -- binary low-rank GEMV y = s1 . U (V^T (s2 . x)), M = 1..4 tokens (sm_100a).
+//
+// Form: "70B en 4GB de VRAM: la compresión neural de 2026, ¿es real?" (nramos.dev),
+// section "1. NanoQuant — sub-1-bit PTQ", bullet "Formulación".  Two chained launches,
+// each one +-1 matrix times a vector with the machinery of the group GEMV:
+//
+//   stage 1: t[m, j] = sum_i V^T[j, i] * s2[i] * x[m, i]       rows r,     columns d_in
+//   stage 2: y[m, i] = s1[i] * sum_j U[i, j] * t[m, j]         rows d_out, columns r
+//
+//  * Every CTA prepares the stage input v (s2 . x, or t) in its shared memory right after
+//    waiting for the previous kernel: one power-of-two scale 2^E per token over the whole
+//    vector (|v| <= 32639 after scaling), int8 planes hi, lo (v = 256 hi + lo) in
+//    B-fragment order and exact per-256-chunk sums of v.
+//  * Warps split the (16-row tile, 256-column superblock) units evenly (warp-level
+//    stream-K) and stream the lanes' 16-byte sign words straight into registers, several
+//    units ahead.  Per k-step a word masked with 0x01010101 << p gives four u8 A-fragment
+//    bytes 2^p * bit (one LOP per four signs); mma.m16n8k32 u8 x s8 accumulates each p in
+//    its own set, and at the tile's end S = sum_p acc_p >> p = sum bit * v exactly.
+//  * sum_k sign * v = 2 S - sum v; the partial of a warp is 2^E (2 S - sum of v over its
+//    superblocks) (times s1 in stage 2); tiles split between warps are finished in fixed
+//    order by the last one to arrive (tile_epilogue), so the result is deterministic.
+//  * Both launches are programmatic dependents; only their first weight loads precede the
+//    wait for the previous kernel.
+#include <cstring>
+#include "lbq_common.cuh"
+#include "lbq_internal.h"
+#include "lbq_group_frag.cuh"
+#include "lbq_ldg.cuh"
+
+namespace lbq {
+
+struct BinStageArgs {
+    const uint8_t* signs;       // kernel sign layout, rows x cpad
+    const uint16_t* x;          // stage 1: [M x cols] activations
+    const uint16_t* s2;         // stage 1: [cols] column scales
+    const float* tin;           // stage 2: [M x cols] stage-1 result
+    float* tout;                // stage 1 output [M x rows]
+    const uint16_t* s1;         // stage 2: [rows] row scales
+    uint16_t* y;                // stage 2 output [M x rows]
+    float* partials;
+    unsigned* counters;
+    int64_t rows, cols, cpad, ksb, n_tiles, total_units, total_warps;
+    int M, maxc;
+    int sp, sv, se, szero;      // shared-memory offsets: planes, chunk sums, exponents, zero chunk
+};
+
+// Byte offset, in a 256-column chunk of a plane row, of column 32p + 16h + 4c + j: the
+// B-fragment bytes (b0: h = 0, b1: h = 1) of k-steps p and p + 1 of lane-group c are one
+// 16-byte piece.
+__device__ __forceinline__ int bin_plane_off(int p, int h, int c) { return 64 * (p >> 1) + 16 * c + 8 * (p & 1) + 4 * h; }
+
+// The lane's 8 consecutive values as q = rint(v * 2^-E) in natural order: hi/lo bytes of
+// elements 0..3 in .x, 4..7 in .y; sum(q) over the whole warp.
+__device__ __forceinline__ PrepOut bin_quantize8(const float (&v)[8], int E) {
+    PrepOut r;
+    r.E = E;
+    const int e1 = max(-126, min(127, -E));
+    const float f1 = ldg_exp2i(e1), f2 = ldg_exp2i(-E - e1);
+    uint32_t h0 = 0, h1 = 0, l0 = 0, l1 = 0;
+    int sum = 0;
+#pragma unroll
+    for (int e = 0; e < 8; e++) {
+        const int q = __float2int_rn((v[e] * f1) * f2);
+        const int h = (q + 128) >> 8;
+        const int l = q - 256 * h;
+        sum += q;
+        const int sh = 8 * (e & 3);
+        if (e < 4) {
+            h0 |= (uint32_t)(h & 0xFF) << sh;
+            l0 |= (uint32_t)(l & 0xFF) << sh;
+        } else {
+            h1 |= (uint32_t)(h & 0xFF) << sh;
+            l1 |= (uint32_t)(l & 0xFF) << sh;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    r.hi = make_uint2(h0, h1);
+    r.lo = make_uint2(l0, l1);
+    r.gsum = sum;
+    return r;
+}
+
+// Lane's 8 stage-input values of token m, columns k0..k0+7 (zero past the last column).
+// The inputs may come from the previous kernel of the stream: read through L2.
+template <bool STAGE2, bool BF16>
+__device__ __forceinline__ void bin_load8(const BinStageArgs& a, int m, int64_t k0, float (&v)[8]) {
+    if (k0 >= a.cols) {
+#pragma unroll
+        for (int e = 0; e < 8; e++) v[e] = 0.0f;
+        return;
+    }
+    if constexpr (STAGE2) {
+        const float4 p = __ldcg(reinterpret_cast<const float4*>(a.tin + (int64_t)m * a.cols + k0));
+        const float4 q = __ldcg(reinterpret_cast<const float4*>(a.tin + (int64_t)m * a.cols + k0 + 4));
+        v[0] = p.x; v[1] = p.y; v[2] = p.z; v[3] = p.w;
+        v[4] = q.x; v[5] = q.y; v[6] = q.z; v[7] = q.w;
+    } else {
+        const uint4 xr = __ldcg(reinterpret_cast<const uint4*>(a.x + (int64_t)m * a.cols + k0));
+        const uint4 sr = __ldg(reinterpret_cast<const uint4*>(a.s2 + k0));
+        const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
+        const uint32_t sw[4] = {sr.x, sr.y, sr.z, sr.w};
+#pragma unroll
+        for (int e = 0; e < 8; e++) {
+            const float xv = to_f32<BF16>((uint16_t)(xw[e / 2] >> (16 * (e & 1))));
+            const float sv = __half2float(__ushort_as_half((uint16_t)(sw[e / 2] >> (16 * (e & 1)))));
+            v[e] = xv * sv;       // exact: a product of two 11- (or 8-) bit significands
+        }
+    }
+}
+
+template <bool STAGE2, int D, bool BF16>
+__global__ void __launch_bounds__(kLdgThreads, 2) k_binlr_ldg(const __grid_constant__ BinStageArgs a) {
+    constexpr int NB = 1;                      // M <= 4: hi/lo planes of 4 tokens in one n-block
+    constexpr int PF = 16;                     // units prefetched into L2 before the wait
+    extern __shared__ __align__(16) uint8_t smem[];
+    griddep_launch_dependents();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int64_t W = a.total_warps, S = a.total_units;
+    const int64_t wid = (int64_t)blockIdx.x * kLdgWarps + warp;
+    const int u_begin = (int)(wid < W ? wid * S / W : S);
+    const int u_end = (int)(wid < W ? (wid + 1) * S / W : S);
+    const bool has_work = u_begin < u_end;
+    const int M = a.M;
+    const int ksb = (int)a.ksb;
+    const uint64_t pol = l2_policy_evict_first();
+
+    int ct = 0, csb = 0;
+    if (has_work) {
+        ct = u_begin / ksb;
+        csb = u_begin % ksb;
+    }
+    const uint8_t* lptr = a.signs + (int64_t)u_begin * 512 + 16 * lane;
+    uint4 wb[D];
+#pragma unroll
+    for (int d = 0; d < D; d++)
+        if (u_begin + d < u_end) wb[d] = ldg_stream(lptr + d * 512, pol);
+    lptr += D * 512;
+    if (lane < PF && u_begin + D + lane < u_end) l2_prefetch_bulk(lptr - 16 * lane + lane * 512, 512);
+    if (threadIdx.x < 16) reinterpret_cast<uint4*>(smem + a.szero)[threadIdx.x] = make_uint4(0, 0, 0, 0);
+    int* maxbits = reinterpret_cast<int*>(smem + a.se) + 4;      // |v| maxima (float bits), M <= 4
+    if (threadIdx.x < 4) maxbits[threadIdx.x] = 0;
+    griddep_wait();
+    __syncthreads();
+
+    // ---- prepare the stage input: per-token maxima, then planes and chunk sums; the chunk
+    // order is rotated by the CTA index so that the CTAs do not all read the same lines
+    const int kch = (int)(a.cpad / kLdgChunk);
+    const int rot = (int)(blockIdx.x % (unsigned)kch);
+    for (int m = 0; m < M; m++) {
+        float mx = 0.0f;
+        for (int cw = warp; cw < kch; cw += kLdgWarps) {
+            const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
+            float v[8];
+            bin_load8<STAGE2, BF16>(a, m, (int64_t)ch * kLdgChunk + 8 * lane, v);
+            mx = fmaxf(mx, warp_max_abs8(v));
+        }
+        if (lane == 0) atomicMax(&maxbits[m], __float_as_int(mx));   // non-negative floats order as ints
+    }
+    __syncthreads();
+    int* expo = reinterpret_cast<int*>(smem + a.se);
+    int* vsum = reinterpret_cast<int*>(smem + a.sv);
+    for (int m = 0; m < M; m++) {
+        const int E = ldg_fixed_point_exponent(__int_as_float(maxbits[m]));
+        if (threadIdx.x == 0) expo[m] = E;
+        int8_t* row_h = reinterpret_cast<int8_t*>(smem + a.sp) + (int64_t)(2 * m) * a.cpad;
+        for (int cw = warp; cw < kch; cw += kLdgWarps) {
+            const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
+            float v[8];
+            bin_load8<STAGE2, BF16>(a, m, (int64_t)ch * kLdgChunk + 8 * lane, v);
+            const PrepOut r = bin_quantize8(v, E);
+            // elements 8 lane + 0..3 and + 4..7: columns 32p + 16h + 4c' + j
+            const int p = lane >> 2, h = (lane & 3) >> 1, c0 = 2 * (lane & 1);
+            int8_t* base = row_h + ch * kLdgChunk;
+            *reinterpret_cast<uint32_t*>(base + bin_plane_off(p, h, c0)) = r.hi.x;
+            *reinterpret_cast<uint32_t*>(base + bin_plane_off(p, h, c0 + 1)) = r.hi.y;
+            *reinterpret_cast<uint32_t*>(base + a.cpad + bin_plane_off(p, h, c0)) = r.lo.x;
+            *reinterpret_cast<uint32_t*>(base + a.cpad + bin_plane_off(p, h, c0 + 1)) = r.lo.y;
+            if (lane == 0) vsum[m * kch + ch] = r.gsum;
+        }
+    }
+    __syncthreads();
+    if (!has_work) return;
+
+    // B-fragment row of this lane (plane g: token g / 2, hi or lo) and its token's sums
+    const bool pv = g < 2 * M;
+    const int8_t* prow = pv ? reinterpret_cast<const int8_t*>(smem + a.sp) + (int64_t)g * a.cpad + 16 * c
+                            : reinterpret_cast<const int8_t*>(smem + a.szero) + 16 * c;
+    const int pstep = pv ? kLdgChunk : 0;
+    const bool tv = c < M;
+    const int* vrow = tv ? vsum + c * kch : reinterpret_cast<const int*>(smem + a.szero);
+    const int vstep = tv ? 1 : 0;
+    const float scale = tv ? ldg_exp2i(expo[c]) : 0.0f;
+
+    int acc[8][4];
+#pragma unroll
+    for (int p = 0; p < 8; p++)
+#pragma unroll
+        for (int e = 0; e < 4; e++) acc[p][e] = 0;
+    int vpart = 0;                                   // sum of v over this warp's superblocks of the tile
+    int tile_first_u = u_begin - csb;
+
+    for (int base = u_begin; base < u_end; base += D) {
+#pragma unroll
+        for (int d = 0; d < D; d++) {
+            const int u = base + d;
+            if (u < u_end) {
+                const uint4 w = wb[d];
+                if (u + D < u_end) {
+                    wb[d] = ldg_stream(lptr, pol);
+                    lptr += 512;
+                }
+                const int8_t* pr = prow + csb * pstep;
+#pragma unroll
+                for (int p = 0; p < 8; p += 2) {
+                    const uint4 bq = *reinterpret_cast<const uint4*>(pr + 64 * (p >> 1));
+#pragma unroll
+                    for (int q = 0; q < 2; q++) {
+                        const uint32_t msk = 0x01010101u << (p + q);
+                        mma_16832_u8s8(acc[p + q], w.x & msk, w.y & msk, w.z & msk, w.w & msk, q ? bq.z : bq.x,
+                                       q ? bq.w : bq.y);
+                    }
+                }
+                vpart += vrow[csb * vstep];
+                if (csb == ksb - 1 || u == u_end - 1) {
+                    // S = sum_p acc_p >> p; columns 2c (hi) and 2c + 1 (lo) of token c
+                    int s[4];
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        int v = 0;
+#pragma unroll
+                        for (int p = 0; p < 8; p++) v += acc[p][e] >> p;
+                        s[e] = v;
+                    }
+                    float part[NB][2];
+                    part[0][0] = scale * (float)(2 * (256 * s[0] + s[1]) - vpart);
+                    part[0][1] = scale * (float)(2 * (256 * s[2] + s[3]) - vpart);
+                    const int64_t row = (int64_t)ct * 16 + g;
+                    if constexpr (STAGE2) {
+                        part[0][0] *= __half2float(__ushort_as_half(a.s1[row]));
+                        part[0][1] *= __half2float(__ushort_as_half(a.s1[row + 8]));
+                    }
+                    const bool full = tile_first_u >= u_begin && csb == ksb - 1;
+                    if constexpr (STAGE2)
+                        tile_epilogue<NB>(part, full, M, a.rows, ct, ct, (int64_t)ct * ksb, ksb, S, W, wid, a.partials,
+                                          a.counters, a.maxc, a.y);
+                    else
+                        tile_epilogue_f32<NB>(part, full, M, a.rows, ct, ct, (int64_t)ct * ksb, ksb, S, W, wid,
+                                              a.partials, a.counters, a.maxc, a.tout);
+#pragma unroll
+                    for (int p = 0; p < 8; p++)
+#pragma unroll
+                        for (int e = 0; e < 4; e++) acc[p][e] = 0;
+                    vpart = 0;
+                    tile_first_u = u + 1;
+                }
+                if (++csb == ksb) {
+                    csb = 0;
+                    ct++;
+                }
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ host side
+struct BinLdgPlan {
+    int64_t units1, units2, warps1, warps2;
+    int grid1, grid2, maxc1, maxc2;
+    size_t part1, part2, t_off, bytes;
+};
+
+static void bin_stage_plan(int64_t rows, int64_t cpad, int64_t& units, int64_t& warps, int& grid, int& maxc) {
+    const int64_t ksb = cpad / kLdgChunk;
+    units = rows / 16 * ksb;
+    constexpr int64_t kMinUnitsPerWarp = 4;
+    grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sm_count() * 2, ceil_div(units, kLdgWarps * kMinUnitsPerWarp)));
+    warps = std::min<int64_t>((int64_t)grid * kLdgWarps, std::max<int64_t>(units, 1));
+    maxc = (int)(ceil_div(ksb * warps, std::max<int64_t>(units, 1)) + 2);
+}
+
+static BinLdgPlan bin_ldg_plan(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
+    BinLdgPlan pl;
+    bin_stage_plan(r, sign_cols_pad(d_in), pl.units1, pl.warps1, pl.grid1, pl.maxc1);
+    bin_stage_plan(d_out, sign_cols_pad(r), pl.units2, pl.warps2, pl.grid2, pl.maxc2);
+    pl.part1 = kCounterBytes;
+    pl.part2 = pl.part1 + al256((size_t)(r / 16 * pl.maxc1 * 16 * M * 4));
+    pl.t_off = pl.part2 + al256((size_t)(d_out / 16 * pl.maxc2 * 16 * M * 4));
+    pl.bytes = pl.t_off + al256((size_t)(M * r * 4));
+    return pl;
+}
+
+static int bin_smem_bytes(int64_t M, int64_t cpad) {
+    // planes [2M][cpad] | chunk sums [M][cpad/256] | exponents and maxima (8 ints) | zero chunk
+    return al16(2 * M * cpad) + al16(M * (cpad / kLdgChunk) * 4) + 32 + 256;
+}
+
+bool gemv_binlr_ldg_supported(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
+    if (M < 1 || M > 4 || d_out % 16 != 0 || r % 32 != 0 || d_in % 32 != 0) return false;
+    // int32 sums: |sum over a tile of bit * v| <= 32639 * columns must stay below 2^30
+    if (d_out / 16 + r / 16 > kMaxTiles || d_in > 32768 || r > 32768) return false;
+    const int budget = 100 * 1024;                 // two CTAs per SM
+    return bin_smem_bytes(M, sign_cols_pad(d_in)) <= budget && bin_smem_bytes(M, sign_cols_pad(r)) <= budget;
+}
+
+size_t gemv_binlr_ldg_ws_bytes(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
+    return bin_ldg_plan(M, d_out, d_in, r).bytes;
+}
+
+template <bool STAGE2, bool BF16>
+static lbq_status launch_bin_stage(const BinStageArgs& a, int grid, int smem, cudaStream_t st) {
+    constexpr int D = 8;
+    constexpr auto kern = k_binlr_ldg<STAGE2, D, BF16>;
+    const lbq_status s = ldg_smem_attr<kern>(100 * 1024);
+    if (s != LBQ_OK) return s;
+    return launch_pdl(kern, grid, kLdgThreads, (size_t)smem, st, a);
+}
+
+lbq_status launch_gemv_binlr_ldg(const void* x, bool bf16, int64_t M, const void* U, const void* Vt, const void* s1,
+                                 const void* s2, int64_t d_out, int64_t d_in, int64_t r, void* y, void* ws,
+                                 size_t ws_bytes, cudaStream_t st) {
+    const BinLdgPlan pl = bin_ldg_plan(M, d_out, d_in, r);
+    if (ws == nullptr || ws_bytes < pl.bytes) return LBQ_ERR_WORKSPACE;
+    char* base = (char*)ws;
+    float* t = (float*)(base + pl.t_off);
+    for (int stage = 0; stage < 2; stage++) {
+        BinStageArgs a;
+        memset(&a, 0, sizeof a);
+        const bool st2 = stage == 1;
+        a.signs = (const uint8_t*)(st2 ? U : Vt);
+        a.rows = st2 ? d_out : r;
+        a.cols = st2 ? r : d_in;
+        a.cpad = sign_cols_pad(a.cols);
+        a.ksb = a.cpad / kLdgChunk;
+        a.n_tiles = a.rows / 16;
+        a.x = (const uint16_t*)x;
+        a.s2 = (const uint16_t*)s2;
+        a.tin = t;
+        a.tout = t;
+        a.s1 = (const uint16_t*)s1;
+        a.y = (uint16_t*)y;
+        a.partials = (float*)(base + (st2 ? pl.part2 : pl.part1));
+        // the two stages' tickets are disjoint ranges of the counter header
+        a.counters = (unsigned*)base + (st2 ? r / 16 : 0);
+        a.total_units = st2 ? pl.units2 : pl.units1;
+        a.total_warps = st2 ? pl.warps2 : pl.warps1;
+        a.M = (int)M;
+        a.maxc = st2 ? pl.maxc2 : pl.maxc1;
+        a.sp = 0;
+        a.sv = al16(2 * M * a.cpad);
+        a.se = a.sv + al16(M * a.ksb * 4);
+        a.szero = a.se + 32;
+        const int smem = bin_smem_bytes(M, a.cpad);
+        const int grid = st2 ? pl.grid2 : pl.grid1;
+        lbq_status s;
+        if (st2) s = bf16 ? launch_bin_stage<true, true>(a, grid, smem, st) : launch_bin_stage<true, false>(a, grid, smem, st);
+        else s = bf16 ? launch_bin_stage<false, true>(a, grid, smem, st) : launch_bin_stage<false, false>(a, grid, smem, st);
+        if (s != LBQ_OK) return s;
+    }
+    return LBQ_OK;
+}
+
+}  // namespace lbq

@@ -37,13 +37,10 @@
 #include "lbq_common.cuh"
 #include "lbq_internal.h"
 #include "lbq_group_frag.cuh"
+#include "lbq_ldg.cuh"
 
 namespace lbq {
 
-constexpr int kLdgWarps = 8;
-constexpr int kLdgThreads = kLdgWarps * 32;
-constexpr int kLdgChunk = 256;                 // k per unit (one superblock)
-constexpr int kLdgPlaneMax = 32639;            // |v| bound so that (v + 128) >> 8 fits in int8
 
 struct LdgProblem {
     const uint8_t* packed;
@@ -89,36 +86,6 @@ struct PrepArgs {
     int count, M;
 };
 
-// Smallest E with maxabs * 2^-E <= kLdgPlaneMax (E = 0 for an all-zero chunk), from the
-// exponent and significand fields (maxabs = m * 2^e, m in [1, 2)).
-__device__ __forceinline__ int ldg_fixed_point_exponent(float maxabs) {
-    if (!(maxabs > 0.0f)) return 0;
-    uint32_t u = __float_as_uint(maxabs);
-    int bias = 0;
-    if ((u >> 23) == 0) {                       // subnormal: scale up exactly by 2^64 first
-        u = __float_as_uint(maxabs * 18446744073709551616.0f);
-        bias = 64;
-    }
-    const int e = (int)(u >> 23) - 127 - bias;
-    const float m = __uint_as_float((u & 0x007FFFFFu) | 0x3F800000u);
-    return e - 14 + (m * 16384.0f > (float)kLdgPlaneMax ? 1 : 0);
-}
-
-// 2^p as a float (exact for every p a normal float holds).
-__device__ __forceinline__ float ldg_exp2i(int p) {
-    if (p >= -126 && p <= 127) return __uint_as_float((uint32_t)(p + 127) << 23);
-    return ldexpf(1.0f, p);
-}
-
-// 16 bytes of streamed weights: read once, so no L1 allocation and evict-first in L2.
-__device__ __forceinline__ uint4 ldg_stream(const void* p, uint64_t pol) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p), "l"(pol));
-    return v;
-}
-
 // NG consecutive fp16 values (NG in 4, 8, 16; 2 * NG-byte aligned) from shared memory.
 template <int NG>
 __device__ __forceinline__ void lds_halves_ldg(const uint16_t* p, uint32_t (&d)[NG / 2]) {
@@ -144,17 +111,6 @@ __device__ __forceinline__ void lds_halves_ldg(const uint16_t* p, uint32_t (&d)[
 // 4(l mod 4).. (even elements) and 16 + 4(l mod 4).. (odd elements) of k-step l / 4.
 // x may have been written by the previous kernel of the stream, so it is read through
 // L2 (ld.global.cg), never through the non-coherent path.
-// Byte offset, inside a 256-wide chunk of a plane row, of the 8 bytes prepared by lane l
-// (elements 8l..8l+7): k-step l / 4, lane-group l mod 4; two consecutive k-steps of a
-// lane-group sit side by side so that one 16-byte load fetches both B fragments.
-__host__ __device__ __forceinline__ int plane_off(int l) { return 64 * (l >> 3) + 16 * (l & 3) + 8 * ((l >> 2) & 1); }
-
-struct PrepOut {
-    uint2 hi, lo;   // this lane's 8 bytes of the hi and lo planes
-    int gsum;       // exact sum of v over the lane's group (valid on the group's first lane)
-    int E;
-};
-
 __device__ __forceinline__ uint4 prep_load(const uint16_t* xc, int lane) {
     return __ldcg(reinterpret_cast<const uint4*>(xc + 8 * lane));
 }
@@ -163,43 +119,9 @@ template <int GROUP, bool BF16>
 __device__ __forceinline__ PrepOut prep_convert(const uint4 raw) {
     const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
     float v[8];
-    float mx = 0.0f;
 #pragma unroll
-    for (int e = 0; e < 8; e++) {
-        v[e] = to_f32<BF16>((uint16_t)(rw[e / 2] >> (16 * (e & 1))));
-        mx = fmaxf(mx, fabsf(v[e]));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    PrepOut r;
-    r.E = ldg_fixed_point_exponent(mx);
-    // v * 2^-E in at most two exact power-of-two multiplications
-    const int e1 = max(-126, min(127, -r.E));
-    const float f1 = ldg_exp2i(e1), f2 = ldg_exp2i(-r.E - e1);
-    uint32_t hev = 0, hod = 0, lev = 0, lod = 0;
-    int sum = 0;
-#pragma unroll
-    for (int e = 0; e < 8; e++) {
-        const int q = __float2int_rn((v[e] * f1) * f2);
-        const int h = (q + 128) >> 8;
-        const int l = q - 256 * h;
-        sum += q;
-        const int sh = 8 * (e >> 1);
-        if (e & 1) {
-            hod |= (uint32_t)(h & 0xFF) << sh;
-            lod |= (uint32_t)(l & 0xFF) << sh;
-        } else {
-            hev |= (uint32_t)(h & 0xFF) << sh;
-            lev |= (uint32_t)(l & 0xFF) << sh;
-        }
-    }
-    constexpr int LPG = GROUP / 8;                 // lanes per group
-#pragma unroll
-    for (int o = 1; o < LPG; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    r.hi = make_uint2(hev, hod);
-    r.lo = make_uint2(lev, lod);
-    r.gsum = sum;                                  // |sum| <= 128 * 32639 < 2^24: exact in fp32
-    return r;
+    for (int e = 0; e < 8; e++) v[e] = to_f32<BF16>((uint16_t)(rw[e / 2] >> (16 * (e & 1))));
+    return prep_quantize8<GROUP / 8>(v, ldg_fixed_point_exponent(warp_max_abs8(v)));
 }
 
 template <int GROUP, bool BF16>
@@ -281,7 +203,9 @@ __global__ void __launch_bounds__(kLdgThreads, CPS)
     using F = IFrag<B>;
     constexpr int KPG = GROUP / 32;                // k-steps per group
     constexpr int NGC = kLdgChunk / GROUP;         // groups per unit
-    constexpr int PF = B == 2 ? 8 : B == 3 ? 5 : B == 4 ? 4 : B == 5 ? 3 : 2;   // units prefetched into L2
+    // units prefetched into L2 before the wait (about 16 KB a warp): HBM keeps streaming
+    // while the activations are prepared
+    constexpr int PF = 16384 / (512 * B);
     extern __shared__ __align__(16) uint8_t smem[];
     griddep_launch_dependents();
 
@@ -366,20 +290,29 @@ __global__ void __launch_bounds__(kLdgThreads, CPS)
     }
     griddep_wait();
     if constexpr (SMEMP) {
-        // this CTA's copy of the prepared activations
-        for (int64_t wi = warp; wi < pa.total_warps; wi += kLdgWarps) {
-            int m;
-            int64_t ch;
-            const PrepSlot& Q = pa.s[prep_task(pa, wi, m, ch)];
-            const PrepOut r = prep_chunk<GROUP, BF16>(Q.x + (int64_t)m * Q.k + ch * kLdgChunk, lane);
-            int8_t* row_h = reinterpret_cast<int8_t*>(smem + Q.sp) + (int64_t)(2 * m) * Q.k + ch * kLdgChunk;
-            *reinterpret_cast<uint2*>(row_h + plane_off(lane)) = r.hi;
-            *reinterpret_cast<uint2*>(row_h + Q.k + plane_off(lane)) = r.lo;
-            constexpr int LPG = GROUP / 8;
-            if (lane % LPG == 0)
-                reinterpret_cast<float*>(smem + Q.sx)[(int64_t)m * (Q.k / GROUP) + ch * (kLdgChunk / GROUP) +
-                                                      lane / LPG] = (float)r.gsum;
-            if (lane == 0) reinterpret_cast<int*>(smem + Q.se)[(int64_t)m * (Q.k / kLdgChunk) + ch] = r.E;
+        // this CTA's copy of the prepared activations: warp w takes chunks w, w + 8, ...
+        // of every token of every slot, rotated by the CTA index so that the CTAs do not all
+        // read the same lines of x at once (no divisions on the way)
+        for (int si = 0; si < pa.count; si++) {
+            const PrepSlot& Q = pa.s[si];
+            const int kch = (int)(Q.k / kLdgChunk);
+            const int k32 = (int)Q.k;
+            const int rot = (int)(blockIdx.x % (unsigned)kch);
+            for (int m = 0; m < M; m++) {
+                const uint16_t* xm = Q.x + (int64_t)m * k32;
+                int8_t* row_h = reinterpret_cast<int8_t*>(smem + Q.sp) + (int64_t)(2 * m) * k32;
+                float* xs = reinterpret_cast<float*>(smem + Q.sx) + m * (k32 / GROUP);
+                int* ex = reinterpret_cast<int*>(smem + Q.se) + m * kch;
+                for (int cw = warp; cw < kch; cw += kLdgWarps) {
+                    const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
+                    const PrepOut r = prep_chunk<GROUP, BF16>(xm + ch * kLdgChunk, lane);
+                    *reinterpret_cast<uint2*>(row_h + ch * kLdgChunk + plane_off(lane)) = r.hi;
+                    *reinterpret_cast<uint2*>(row_h + k32 + ch * kLdgChunk + plane_off(lane)) = r.lo;
+                    constexpr int LPG = GROUP / 8;
+                    if (lane % LPG == 0) xs[ch * (kLdgChunk / GROUP) + lane / LPG] = (float)r.gsum;
+                    if (lane == 0) ex[ch] = r.E;
+                }
+            }
         }
     }
     __syncthreads();
@@ -558,8 +491,11 @@ static LdgPlan plan_ldg(const int64_t* n, const int64_t* k, int count, int cps) 
         pl.total_tiles += n_tiles;
         max_ksb = std::max(max_ksb, ksb);
     }
+    // at least kMinUnitsPerWarp units a warp: small products then split each tile over
+    // fewer warps (cheaper fixups) and still keep several units in flight per warp
+    constexpr int64_t kMinUnitsPerWarp = 4;
     pl.grid = (int)std::max<int64_t>(
-        1, std::min<int64_t>((int64_t)sm_count() * cps, ceil_div(pl.total_units, (int64_t)kLdgWarps)));
+        1, std::min<int64_t>((int64_t)sm_count() * cps, ceil_div(pl.total_units, kLdgWarps * kMinUnitsPerWarp)));
     // no more warps than units: every participating warp then owns at least one unit,
     // so each warp counted as a contributor to a tile also arrives at its ticket
     pl.total_warps = std::min<int64_t>((int64_t)pl.grid * kLdgWarps, std::max<int64_t>(pl.total_units, 1));
@@ -571,7 +507,6 @@ static LdgPlan plan_ldg(const int64_t* n, const int64_t* k, int count, int cps) 
 
 // Workspace: ticket header, partial tiles, then per product the planes [2M][k], the
 // group sums [M][k/32] (enough for every group size) and the exponents [M][k/256].
-static size_t al256(size_t v) { return (v + 255) / 256 * 256; }
 
 static size_t prep_bytes(int64_t k, int64_t M) {
     return al256((size_t)(2 * M * k)) + al256((size_t)(M * (k / 32) * 4)) + al256((size_t)(M * (k / kLdgChunk) * 4));
@@ -595,36 +530,9 @@ bool gemv_group_ldg_supported(int64_t M, int64_t n, int64_t k, int bits, int gro
     return n / 16 <= kMaxTiles && k <= ((int64_t)1 << 22);
 }
 
-template <class Kern, class... Args>
-static lbq_status launch_pdl(Kern kern, int grid, int threads, size_t smem, cudaStream_t st, const Args&... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, args...) != cudaSuccess) return LBQ_ERR_CUDA;
-    return launch_status();
-}
-
 // Shared memory a CTA may spend on prepared activations (two CTAs per SM share 228 KB).
 static int ldg_smem_budget(int cps) { return cps == 2 ? 100 * 1024 : 200 * 1024; }
 
-template <auto KERN>
-static lbq_status ldg_smem_attr(int bytes) {
-    static bool set[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return LBQ_ERR_CUDA;
-    if (dev >= 0 && dev < 64 && set[dev]) return LBQ_OK;
-    if (cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
-        return LBQ_ERR_CUDA;
-    if (dev >= 0 && dev < 64) set[dev] = true;
-    return LBQ_OK;
-}
 
 template <int B, int GROUP, int NB>
 static lbq_status launch_ldg_inst(int grid, bool smemp, bool bf16, int smem, cudaStream_t st, const LdgArgs& args,
@@ -661,7 +569,6 @@ static lbq_status launch_ldg_b(int group, int NB, int grid, bool smemp, bool bf1
     return launch_ldg_nb<B, 128>(NB, grid, smemp, bf16, smem, st, args, prep);
 }
 
-static int al16(int64_t v) { return (int)((v + 15) / 16 * 16); }
 
 lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count, bool bf16, int64_t M, int bits,
                                        int group, void* ws, size_t ws_bytes, cudaStream_t st) {

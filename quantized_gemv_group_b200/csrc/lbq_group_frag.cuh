@@ -41,11 +41,15 @@ struct IFrag {
 // resets the ticket.  The row block's units are [first_u, first_u + units_per_rb) of
 // the launch's unit list, split evenly over NC CTAs (start(b) = b * S_total / NC);
 // `gtile` indexes the launch-wide ticket and partial arrays, `tile` the rows of y.
-template <int NB>
-__device__ __forceinline__ void tile_epilogue(const float (&acc)[NB][2], bool full, int M, int64_t n, int64_t tile,
-                                              int64_t gtile, int64_t first_u, int64_t units_per_rb, int64_t S_total,
-                                              int64_t NC, int64_t cta, float* __restrict__ partials,
-                                              unsigned* __restrict__ counters, int maxc, uint16_t* __restrict__ y) {
+// Y is uint16_t (fp16 output) or float.
+__device__ __forceinline__ void store_out(uint16_t* p, float v) { *p = from_f32<false>(v); }
+__device__ __forceinline__ void store_out(float* p, float v) { *p = v; }
+
+template <int NB, class Y>
+__device__ __forceinline__ void tile_epilogue_any(const float (&acc)[NB][2], bool full, int M, int64_t n, int64_t tile,
+                                                  int64_t gtile, int64_t first_u, int64_t units_per_rb,
+                                                  int64_t S_total, int64_t NC, int64_t cta, float* __restrict__ partials,
+                                                  unsigned* __restrict__ counters, int maxc, Y* __restrict__ y) {
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
     const int64_t row_g = tile * 16 + g;
@@ -54,8 +58,8 @@ __device__ __forceinline__ void tile_epilogue(const float (&acc)[NB][2], bool fu
         for (int nb = 0; nb < NB; nb++) {
             const int tok = 4 * nb + c;
             if (tok < M) {
-                y[(int64_t)tok * n + row_g] = from_f32<false>(acc[nb][0]);
-                y[(int64_t)tok * n + row_g + 8] = from_f32<false>(acc[nb][1]);
+                store_out(y + (int64_t)tok * n + row_g, acc[nb][0]);
+                store_out(y + (int64_t)tok * n + row_g + 8, acc[nb][1]);
             }
         }
         return;
@@ -84,14 +88,41 @@ __device__ __forceinline__ void tile_epilogue(const float (&acc)[NB][2], bool fu
     if (old == (unsigned)(count - 1)) {
         __threadfence();
         const float* p0 = partials + (gtile * maxc) * (int64_t)(16 * M);
+        // The slots' loads are independent: issue them in batches of 8 so that their L2
+        // latencies overlap, and add the slots in their fixed order.
         for (int e = lane; e < 16 * M; e += 32) {
             float s = 0.0f;
-            for (int sl = 0; sl < count; sl++) s += __ldcg(p0 + sl * (int64_t)(16 * M) + e);
-            y[(int64_t)(e / 16) * n + tile * 16 + (e % 16)] = from_f32<false>(s);
+            int sl = 0;
+            for (; sl + 8 <= count; sl += 8) {
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; j++) v[j] = __ldcg(p0 + (sl + j) * (int64_t)(16 * M) + e);
+#pragma unroll
+                for (int j = 0; j < 8; j++) s += v[j];
+            }
+            for (; sl < count; sl++) s += __ldcg(p0 + sl * (int64_t)(16 * M) + e);
+            store_out(y + (int64_t)(e / 16) * n + tile * 16 + (e % 16), s);
         }
         __syncwarp();
         if (lane == 0) counters[gtile] = 0u;
     }
+}
+
+template <int NB>
+__device__ __forceinline__ void tile_epilogue(const float (&acc)[NB][2], bool full, int M, int64_t n, int64_t tile,
+                                              int64_t gtile, int64_t first_u, int64_t units_per_rb, int64_t S_total,
+                                              int64_t NC, int64_t cta, float* __restrict__ partials,
+                                              unsigned* __restrict__ counters, int maxc, uint16_t* __restrict__ y) {
+    tile_epilogue_any<NB, uint16_t>(acc, full, M, n, tile, gtile, first_u, units_per_rb, S_total, NC, cta, partials,
+                                    counters, maxc, y);
+}
+template <int NB>
+__device__ __forceinline__ void tile_epilogue_f32(const float (&acc)[NB][2], bool full, int M, int64_t n,
+                                                  int64_t tile, int64_t gtile, int64_t first_u, int64_t units_per_rb,
+                                                  int64_t S_total, int64_t NC, int64_t cta, float* __restrict__ partials,
+                                                  unsigned* __restrict__ counters, int maxc, float* __restrict__ y) {
+    tile_epilogue_any<NB, float>(acc, full, M, n, tile, gtile, first_u, units_per_rb, S_total, NC, cta, partials,
+                                 counters, maxc, y);
 }
 
 }  // namespace lbq

@@ -89,6 +89,13 @@ lbq_status launch_gemm_binlr_tc(const void* x, bool bf16, int64_t M, const void*
                                 const void* s2, int64_t d_out, int64_t d_in, int64_t r, void* y, void* ws,
                                 size_t ws_bytes, cudaStream_t st);
 
+// Binary low-rank GEMV streaming the signs into registers (M <= 4, sign kernel layout).
+bool gemv_binlr_ldg_supported(int64_t M, int64_t d_out, int64_t d_in, int64_t r);
+size_t gemv_binlr_ldg_ws_bytes(int64_t M, int64_t d_out, int64_t d_in, int64_t r);
+lbq_status launch_gemv_binlr_ldg(const void* x, bool bf16, int64_t M, const void* U, const void* Vt, const void* s1,
+                                 const void* s2, int64_t d_out, int64_t d_in, int64_t r, void* y, void* ws,
+                                 size_t ws_bytes, cudaStream_t st);
+
 // Binary low-rank GEMV (M <= 16).
 size_t gemv_binlr_ws_bytes(int64_t M, int64_t d_out, int64_t d_in, int64_t r, lbq_layout layout);
 lbq_status launch_gemv_binlr(const void* x, bool bf16, int64_t M, const void* U, const void* Vt, const void* s1,
