@@ -29,6 +29,9 @@
 
 namespace lbq {
 
+constexpr int kBinWarpsPerCta = 16;          // one CTA per SM: the stage input is prepared once per SM
+constexpr int kBinThreads = kBinWarpsPerCta * 32;
+
 struct BinStageArgs {
     const uint8_t* signs;       // kernel sign layout, rows x cpad
     const uint16_t* x;          // stage 1: [M x cols] activations
@@ -110,7 +113,7 @@ __device__ __forceinline__ void bin_load8(const BinStageArgs& a, int m, int64_t 
 }
 
 template <bool STAGE2, int D, bool BF16>
-__global__ void __launch_bounds__(kLdgThreads, 2) k_binlr_ldg(const __grid_constant__ BinStageArgs a) {
+__global__ void __launch_bounds__(kBinThreads, 1) k_binlr_ldg(const __grid_constant__ BinStageArgs a) {
     constexpr int NB = 1;                      // M <= 4: hi/lo planes of 4 tokens in one n-block
     constexpr int PF = 16;                     // units prefetched into L2 before the wait
     extern __shared__ __align__(16) uint8_t smem[];
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(kLdgThreads, 2) k_binlr_ldg(const __grid_const
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
     const int64_t W = a.total_warps, S = a.total_units;
-    const int64_t wid = (int64_t)blockIdx.x * kLdgWarps + warp;
+    const int64_t wid = (int64_t)blockIdx.x * kBinWarpsPerCta + warp;
     const int u_begin = (int)(wid < W ? wid * S / W : S);
     const int u_end = (int)(wid < W ? (wid + 1) * S / W : S);
     const bool has_work = u_begin < u_end;
@@ -151,7 +154,7 @@ __global__ void __launch_bounds__(kLdgThreads, 2) k_binlr_ldg(const __grid_const
     const int rot = (int)(blockIdx.x % (unsigned)kch);
     for (int m = 0; m < M; m++) {
         float mx = 0.0f;
-        for (int cw = warp; cw < kch; cw += kLdgWarps) {
+        for (int cw = warp; cw < kch; cw += kBinWarpsPerCta) {
             const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
             float v[8];
             bin_load8<STAGE2, BF16>(a, m, (int64_t)ch * kLdgChunk + 8 * lane, v);
@@ -166,7 +169,7 @@ __global__ void __launch_bounds__(kLdgThreads, 2) k_binlr_ldg(const __grid_const
         const int E = ldg_fixed_point_exponent(__int_as_float(maxbits[m]));
         if (threadIdx.x == 0) expo[m] = E;
         int8_t* row_h = reinterpret_cast<int8_t*>(smem + a.sp) + (int64_t)(2 * m) * a.cpad;
-        for (int cw = warp; cw < kch; cw += kLdgWarps) {
+        for (int cw = warp; cw < kch; cw += kBinWarpsPerCta) {
             const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
             float v[8];
             bin_load8<STAGE2, BF16>(a, m, (int64_t)ch * kLdgChunk + 8 * lane, v);
@@ -276,8 +279,8 @@ static void bin_stage_plan(int64_t rows, int64_t cpad, int64_t& units, int64_t& 
     const int64_t ksb = cpad / kLdgChunk;
     units = rows / 16 * ksb;
     constexpr int64_t kMinUnitsPerWarp = 4;
-    grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sm_count() * 2, ceil_div(units, kLdgWarps * kMinUnitsPerWarp)));
-    warps = std::min<int64_t>((int64_t)grid * kLdgWarps, std::max<int64_t>(units, 1));
+    grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sm_count(), ceil_div(units, kBinWarpsPerCta * kMinUnitsPerWarp)));
+    warps = std::min<int64_t>((int64_t)grid * kBinWarpsPerCta, std::max<int64_t>(units, 1));
     maxc = (int)(ceil_div(ksb * warps, std::max<int64_t>(units, 1)) + 2);
 }
 
@@ -301,7 +304,7 @@ bool gemv_binlr_ldg_supported(int64_t M, int64_t d_out, int64_t d_in, int64_t r)
     if (M < 1 || M > 4 || d_out % 16 != 0 || r % 32 != 0 || d_in % 32 != 0) return false;
     // int32 sums: |sum over a tile of bit * v| <= 32639 * columns must stay below 2^30
     if (d_out / 16 + r / 16 > kMaxTiles || d_in > 32768 || r > 32768) return false;
-    const int budget = 100 * 1024;                 // two CTAs per SM
+    const int budget = 200 * 1024;                 // one CTA per SM
     return bin_smem_bytes(M, sign_cols_pad(d_in)) <= budget && bin_smem_bytes(M, sign_cols_pad(r)) <= budget;
 }
 
@@ -313,9 +316,9 @@ template <bool STAGE2, bool BF16>
 static lbq_status launch_bin_stage(const BinStageArgs& a, int grid, int smem, cudaStream_t st) {
     constexpr int D = 8;
     constexpr auto kern = k_binlr_ldg<STAGE2, D, BF16>;
-    const lbq_status s = ldg_smem_attr<kern>(100 * 1024);
+    const lbq_status s = ldg_smem_attr<kern>(200 * 1024);
     if (s != LBQ_OK) return s;
-    return launch_pdl(kern, grid, kLdgThreads, (size_t)smem, st, a);
+    return launch_pdl(kern, grid, kBinThreads, (size_t)smem, st, a);
 }
 
 lbq_status launch_gemv_binlr_ldg(const void* x, bool bf16, int64_t M, const void* U, const void* Vt, const void* s1,

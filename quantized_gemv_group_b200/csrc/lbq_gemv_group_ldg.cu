@@ -193,11 +193,12 @@ __device__ __forceinline__ T ld_prep(const T* p) {
 }
 
 // ------------------------------------------------------------------ GEMV
-// D units in flight per warp; CPS resident CTAs per SM (2: up to 128 registers a thread);
+// D units in flight per warp; NW warps per CTA, one CTA per SM (NW = 16: up to 128 registers
+// a thread, NW = 8: up to 255);
 // SMEMP: every CTA prepares the activations itself, in its shared memory, right after
 // waiting for the previous kernel (else they come from k_gemv_prep via L2).
-template <int B, int GROUP, int NB, int D, int CPS, bool SMEMP, bool BF16>
-__global__ void __launch_bounds__(kLdgThreads, CPS)
+template <int B, int GROUP, int NB, int D, int NW, bool SMEMP, bool BF16>
+__global__ void __launch_bounds__(NW * 32, 1)
     k_gemv_group_ldg(const __grid_constant__ LdgArgs a, const __grid_constant__ PrepArgs pa) {
     using G = GroupGeom<B>;
     using F = IFrag<B>;
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(kLdgThreads, CPS)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
     const int64_t W = a.total_warps, S = a.total_units;
-    const int64_t wid = (int64_t)blockIdx.x * kLdgWarps + warp;
+    const int64_t wid = (int64_t)blockIdx.x * NW + warp;
     // warps past the W that share the list (grid * 8 may exceed it) take no units;
     // unit indices fit 32 bits (the host caps the list)
     const int u_begin = (int)(wid < W ? wid * S / W : S);
@@ -303,7 +304,7 @@ __global__ void __launch_bounds__(kLdgThreads, CPS)
                 int8_t* row_h = reinterpret_cast<int8_t*>(smem + Q.sp) + (int64_t)(2 * m) * k32;
                 float* xs = reinterpret_cast<float*>(smem + Q.sx) + m * (k32 / GROUP);
                 int* ex = reinterpret_cast<int*>(smem + Q.se) + m * kch;
-                for (int cw = warp; cw < kch; cw += kLdgWarps) {
+                for (int cw = warp; cw < kch; cw += NW) {
                     const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
                     const PrepOut r = prep_chunk<GROUP, BF16>(xm + ch * kLdgChunk, lane);
                     *reinterpret_cast<uint2*>(row_h + ch * kLdgChunk + plane_off(lane)) = r.hi;
@@ -462,18 +463,19 @@ __global__ void __launch_bounds__(kLdgThreads, CPS)
 }
 
 // ------------------------------------------------------------------ host side
-// Units in flight per warp and CTAs per SM.  Two CTAs (16 warps, <= 128 registers a
-// thread) with about 12 x 16 bytes in flight per lane where the registers allow it;
-// otherwise one CTA of 8 warps with twice the depth.  Either way each SM keeps about
-// 96 KB of weights in flight, twice what 1 us of HBM latency at full rate needs.
+// Units in flight per warp and warps per CTA (one CTA per SM, so that the activations are
+// prepared once per SM).  16 warps (<= 128 registers a thread) with about 12 x 16 bytes in
+// flight per lane where the registers allow it; otherwise 8 warps with twice the depth.
+// Either way each SM keeps about 96 KB of weights in flight, twice what 1 us of HBM
+// latency at full rate needs.
 struct LdgShape {
-    int D, CPS;
+    int D, NW;
 };
 constexpr LdgShape ldg_shape(int bits, int group, int nb) {
-    const int d = bits == 2 ? 5 : bits == 3 ? 3 : bits == 4 ? 3 : 2;
-    const bool two = nb == 1 && !(group == 32 && bits >= 5);
-    if (two) return {(group == 32 && bits == 4) ? 2 : d, 2};
-    return {nb >= 4 ? d + d / 2 : 2 * d, 1};
+    const int d = bits == 2 ? 4 : bits == 3 ? 3 : bits == 4 ? 3 : 2;
+    const bool wide = nb == 1 && !(group == 32 && bits >= 5);
+    if (wide) return {(group == 32 && bits == 4) ? 2 : d, 16};
+    return {nb >= 4 ? d + d / 2 : 2 * d, 8};
 }
 
 struct LdgPlan {
@@ -481,7 +483,7 @@ struct LdgPlan {
     int grid = 1, maxc = 2;
 };
 
-static LdgPlan plan_ldg(const int64_t* n, const int64_t* k, int count, int cps) {
+static LdgPlan plan_ldg(const int64_t* n, const int64_t* k, int count, int nw) {
     LdgPlan pl;
     int64_t max_ksb = 1;
     for (int i = 0; i < count; i++) {
@@ -495,10 +497,10 @@ static LdgPlan plan_ldg(const int64_t* n, const int64_t* k, int count, int cps) 
     // fewer warps (cheaper fixups) and still keep several units in flight per warp
     constexpr int64_t kMinUnitsPerWarp = 4;
     pl.grid = (int)std::max<int64_t>(
-        1, std::min<int64_t>((int64_t)sm_count() * cps, ceil_div(pl.total_units, kLdgWarps * kMinUnitsPerWarp)));
+        1, std::min<int64_t>((int64_t)sm_count(), ceil_div(pl.total_units, nw * kMinUnitsPerWarp)));
     // no more warps than units: every participating warp then owns at least one unit,
     // so each warp counted as a contributor to a tile also arrives at its ticket
-    pl.total_warps = std::min<int64_t>((int64_t)pl.grid * kLdgWarps, std::max<int64_t>(pl.total_units, 1));
+    pl.total_warps = std::min<int64_t>((int64_t)pl.grid * nw, std::max<int64_t>(pl.total_units, 1));
     // warps that share one tile: the slices are floor(w S / W), so a window of ksb units
     // meets at most ceil(ksb W / S) + 1 of them; one more slot of margin
     pl.maxc = (int)(ceil_div(max_ksb * pl.total_warps, std::max<int64_t>(pl.total_units, 1)) + 2);
@@ -512,9 +514,9 @@ static size_t prep_bytes(int64_t k, int64_t M) {
     return al256((size_t)(2 * M * k)) + al256((size_t)(M * (k / 32) * 4)) + al256((size_t)(M * (k / kLdgChunk) * 4));
 }
 
-// The workspace is sized for the larger grid (two CTAs per SM), which every shape fits.
+// The workspace is sized for the larger warp count (16 a CTA), which every shape fits.
 size_t gemv_group_ldg_ws_bytes_multi(const int64_t* n, const int64_t* k, int count, int64_t M) {
-    const LdgPlan pl = plan_ldg(n, k, count, 2);
+    const LdgPlan pl = plan_ldg(n, k, count, 16);
     size_t b = kCounterBytes + al256((size_t)(pl.total_tiles * pl.maxc * 16 * M * 4));
     for (int i = 0; i < count; i++) b += prep_bytes(k[i], M);
     return b + 256;                                      // zero chunk
@@ -531,7 +533,7 @@ bool gemv_group_ldg_supported(int64_t M, int64_t n, int64_t k, int bits, int gro
 }
 
 // Shared memory a CTA may spend on prepared activations (two CTAs per SM share 228 KB).
-static int ldg_smem_budget(int cps) { return cps == 2 ? 100 * 1024 : 200 * 1024; }
+constexpr int kLdgSmemBudget = 200 * 1024;     // one CTA per SM
 
 
 template <int B, int GROUP, int NB>
@@ -540,16 +542,17 @@ static lbq_status launch_ldg_inst(int grid, bool smemp, bool bf16, int smem, cud
     constexpr LdgShape sh = ldg_shape(B, GROUP, NB);
     if constexpr (NB == 1) {
         if (smemp) {
-            constexpr auto kb = k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.CPS, true, true>;
-            constexpr auto kh = k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.CPS, true, false>;
-            const lbq_status s = bf16 ? ldg_smem_attr<kb>(ldg_smem_budget(sh.CPS))
-                                      : ldg_smem_attr<kh>(ldg_smem_budget(sh.CPS));
+            constexpr auto kb = k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.NW, true, true>;
+            constexpr auto kh = k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.NW, true, false>;
+            const lbq_status s = bf16 ? ldg_smem_attr<kb>(kLdgSmemBudget) : ldg_smem_attr<kh>(kLdgSmemBudget);
             if (s != LBQ_OK) return s;
-            return launch_pdl(bf16 ? kb : kh, grid, kLdgThreads, (size_t)smem, st, args, prep);
+            return launch_pdl(bf16 ? kb : kh, grid, sh.NW * 32, (size_t)smem, st, args, prep);
         }
     }
-    return launch_pdl(k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.CPS, false, false>, grid, kLdgThreads, (size_t)smem,
-                      st, args, prep);
+    constexpr auto kg = k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.NW, false, false>;
+    const lbq_status s = ldg_smem_attr<kg>(kLdgSmemBudget);
+    if (s != LBQ_OK) return s;
+    return launch_pdl(kg, grid, sh.NW * 32, (size_t)smem, st, args, prep);
 }
 
 template <int B, int GROUP>
@@ -579,7 +582,7 @@ lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count,
     }
     const int NB = (int)((2 * M + 7) / 8);
     const LdgShape shape = ldg_shape(bits, group, NB);
-    const LdgPlan pl = plan_ldg(n, k, count, shape.CPS);
+    const LdgPlan pl = plan_ldg(n, k, count, shape.NW);
     if (pl.total_units == 0) return LBQ_OK;
     if (ws == nullptr || ws_bytes < gemv_group_ldg_ws_bytes_multi(n, k, count, M)) return LBQ_ERR_WORKSPACE;
     if (pl.total_tiles > kMaxTiles || pl.total_units >= ((int64_t)1 << 31)) return LBQ_ERR_UNSUPPORTED;
@@ -642,8 +645,8 @@ lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count,
 
     // prepared activations in each CTA's shared memory when they fit, else one prep launch;
     // the scale/zero rings follow them (or start the shared memory)
-    const int ring = kLdgWarps * kScaleRing * scale_slot_bytes(group);
-    const bool smemp = NB == 1 && soff + ring + 256 <= ldg_smem_budget(shape.CPS);
+    const int ring = shape.NW * kScaleRing * scale_slot_bytes(group);
+    const bool smemp = NB == 1 && soff + ring + 256 <= kLdgSmemBudget;
     args.sring = smemp ? al16(soff) : 0;
     args.szero = args.sring + ring;
     const int smem = args.szero + 256;

@@ -6,8 +6,6 @@
 
 namespace lbq {
 
-constexpr int kLdgWarps = 8;
-constexpr int kLdgThreads = kLdgWarps * 32;
 constexpr int kLdgChunk = 256;                 // k per unit (one superblock)
 constexpr int kLdgPlaneMax = 32639;            // |v| bound so that (v + 128) >> 8 fits in int8
 
