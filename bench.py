@@ -590,6 +590,10 @@ def run_prefill(args, dev):
     stream = torch.cuda.Stream(device=dev)
     Ms = [1, 4, 16, 64, 256, 1024]
     shapes = [("gate_up", 28672, 8192), ("down", 8192, 28672)]
+    if args.prefill_m:
+        Ms = [int(v) for v in args.prefill_m.split(",")]
+    if args.prefill_shape:
+        shapes = [sh for sh in shapes if sh[0] in args.prefill_shape.split(",")]
     reps = 8
     cases = []
     for name, n, k in shapes:
@@ -682,6 +686,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["prefill"], default="block")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="print per-linear device times to stderr and exit")
+    ap.add_argument("--prefill-m", default="", help="prefill sweep: comma-separated token counts (default all)")
+    ap.add_argument("--prefill-shape", default="", help="prefill sweep: gate_up and/or down (default both)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     _, _, local = _rank_info()

@@ -55,16 +55,6 @@ lbq_status launch_gemv_group(const void* x, bool bf16, int64_t M, const void* pa
                              const void* zeros, int64_t n, int64_t k, int bits, int group, lbq_layout layout,
                              void* y, void* ws, size_t ws_bytes, cudaStream_t st);
 
-// TMA-pipelined group GEMV (kernel layout, M <= 16, k % 256 == 0, (k/group) % 8 == 0).
-bool gemv_group_tma_supported(int64_t M, int64_t n, int64_t k, int bits, int group);
-size_t gemv_group_tma_ws_bytes(int64_t M, int64_t n, int64_t k);
-size_t gemv_group_tma_ws_bytes_multi(const int64_t* n, const int64_t* k, int count, int64_t M);
-lbq_status launch_gemv_group_tma_multi(const lbq_gemv_problem* probs, int count, bool bf16, int64_t M, int bits,
-                                       int group, void* ws, size_t ws_bytes, cudaStream_t st);
-lbq_status launch_gemv_group_tma(const void* x, bool bf16, int64_t M, const void* packed, const void* scales,
-                                 const void* zeros, int64_t n, int64_t k, int bits, int group, void* y, void* ws,
-                                 size_t ws_bytes, cudaStream_t st);
-
 // Group GEMV with weights streamed into registers (M <= 16, kernel layout).
 bool gemv_group_ldg_supported(int64_t M, int64_t n, int64_t k, int bits, int group);
 size_t gemv_group_ldg_ws_bytes(int64_t M, int64_t n, int64_t k);
