@@ -44,10 +44,11 @@ METRIC = "low-bit GEMV weight GB/s (% of B200 HBM peak); 70B-shaped decode steps
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 
-# dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel,
-# from the ncu captures summarised under profiles/ (None until captured for the
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the step's kernel (mean over
+# the step's launches), from the ncu capture summarised in
+# profiles/k_gemv_group_ldg__llama2_70b_block_int4_g64_m1.md (None: not captured for the
 # current kernel version).
-NCU_TRAFFIC = {"block": None, "sweep80": None, "binlr": None}
+NCU_TRAFFIC = {"block": (481.64e6 + 0.54e6) / 4, "sweep80": None, "binlr": None}
 
 
 # ---------------------------------------------------------------- helpers
@@ -328,7 +329,8 @@ class BinlrWorkload:
                    for (o, i), r in zip(self.shapes, self.ranks))
         self.ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
         self.bytes_per_step = sum(wl.binlr_algorithmic_bytes(o, i, r, M) for (o, i), r in zip(self.shapes, self.ranks))
-        self.launches_per_step = 5 * len(self.shapes)
+        # two launches per product (the register-streaming path for M <= 4), else five
+        self.launches_per_step = (2 if M <= 4 else 5) * len(self.shapes)
         torch.cuda.synchronize()
 
     def run_copy(self, c, xs=None, ys=None):
@@ -513,8 +515,11 @@ def run_gpu(args, dev):
             "config": wk.config(),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": NCU_TRAFFIC.get(wk.name),
-                         "peak_kind": peak_kind,
-                         "note": "algorithmic bytes per step / device time of the step's kernels"},
+                         "algorithmic_bytes_per_launch": wk.bytes_per_step / wk.launches_per_step,
+                         "launches_per_step": wk.launches_per_step, "peak_kind": peak_kind,
+                         "note": "every launch of the step is the same kernel: algorithmic bytes per launch / "
+                                 "mean launch time (CUDA events over the timed replays); traffic per launch "
+                                 "from ncu"},
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": wk.launches_per_step * args.steps,
             "clocks": clocks}
