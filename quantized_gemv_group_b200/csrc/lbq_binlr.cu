@@ -38,7 +38,6 @@ struct BinWs {
     size_t bytes;
 };
 
-static size_t al256(size_t v) { return (v + 255) / 256 * 256; }
 
 static BinWs bin_ws(void* base, int64_t M, int64_t d_out, int64_t d_in, int64_t r, lbq_layout layout) {
     BinWs w{};

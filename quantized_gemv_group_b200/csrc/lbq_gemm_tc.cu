@@ -31,11 +31,12 @@
 namespace lbq {
 
 constexpr int kGemmDq = 8;                         // dequant warps, one per 16-row tile
+constexpr int kGemmDq0 = 2;                        // first dequant warp
 constexpr int kGemmThreads = (3 + kGemmDq) * 32;   // codes producer, MMA, dequant x8, x producer
 constexpr int kXWarp = 2 + kGemmDq;
 constexpr int kPiece = 64;                         // k per A piece = one 128-byte swizzle row
 constexpr int kCodeStages = 3;
-constexpr int kXStages = 3;
+constexpr int kMaxXStages = 8;                     // activation ring depth: as deep as shared memory allows
 constexpr int kAStages = 2;
 constexpr int kGScaleBox = 8;                      // groups per scale/zero box
 constexpr int kGScaleTile = 128 * kGScaleBox * 2;  // bytes of one 128 x 8 fp16 box
@@ -44,9 +45,9 @@ constexpr int kAStageBytes = 128 * kPiece * 2;     // 16 KB
 // B = 2..6: group codes with scale/zero boxes; B = 1: a +-1 sign matrix (no scales).
 struct GemmSmem {
     int x, a, codes, code_stage, sc, zr, bars, bytes;
-    __host__ __device__ GemmSmem(int B, int NT) {
+    __host__ __device__ GemmSmem(int B, int NT, int XS) {
         x = 0;                                           // every stage 1024-byte aligned
-        a = x + kXStages * NT * 128;
+        a = x + XS * NT * 128;
         codes = a + kAStages * kAStageBytes;
         code_stage = 4096 * B + (B > 1 ? 2 * kGScaleTile : 0);
         sc = 4096 * B;                                   // offsets inside a code stage
@@ -64,6 +65,9 @@ struct GemmArgs {
     uint16_t* y;           // fp16 [M x ldy]
     int64_t n, ksb, M, ldy;    // rows of A, k superblocks, tokens, output row stride
     unsigned* err;
+    float* partials;           // split-K: [tile][split][128][NT] fp32 (splits > 1)
+    unsigned* counters;        // split-K tickets, one per output tile (zero between calls)
+    int xs, splits;            // activation ring depth, k slices per output tile
 };
 
 // Byte offset of the 16-byte chunk (row r, k-octet k8) in a 128-row x 64-k fp16 piece,
@@ -126,20 +130,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
     constexpr uint32_t kTmemCols = NT < 32 ? 32 : NT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-    const GemmSmem S(B, NT);
+    const int XS = a.xs;
+    const GemmSmem S(B, NT, XS);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S.bars);
-    // c_full[3] c_empty[3] x_full[3] x_empty[3] a_full[2] a_empty[2] d_full | tmem address | abort
+    // c_full[3] c_empty[3] x_full[8] x_empty[8] a_full[2] a_empty[2] d_full | tmem address |
+    // abort flag | split ticket result
     const uint32_t c_full0 = smem_u32(&bars[0]), c_empty0 = smem_u32(&bars[3]);
-    const uint32_t x_full0 = smem_u32(&bars[6]), x_empty0 = smem_u32(&bars[9]);
-    const uint32_t a_full0 = smem_u32(&bars[12]), a_empty0 = smem_u32(&bars[14]);
-    const uint32_t d_full = smem_u32(&bars[16]);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[17]);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[18]);
+    const uint32_t x_full0 = smem_u32(&bars[6]), x_empty0 = smem_u32(&bars[6 + kMaxXStages]);
+    const uint32_t a_full0 = smem_u32(&bars[6 + 2 * kMaxXStages]), a_empty0 = smem_u32(&bars[8 + 2 * kMaxXStages]);
+    const uint32_t d_full = smem_u32(&bars[10 + 2 * kMaxXStages]);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[11 + 2 * kMaxXStages]);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[12 + 2 * kMaxXStages]);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(&bars[13 + 2 * kMaxXStages]);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n_tt = (a.M + NT - 1) / NT;
-    const int64_t rb = blockIdx.x / n_tt, tt = blockIdx.x % n_tt;
-    const int64_t KSB = a.ksb;
+    const int splits = a.splits;
+    const int64_t tile_id = blockIdx.x / splits;      // output tile (row block, token tile)
+    const int ks = (int)(blockIdx.x % splits);        // k slice of this CTA
+    const int64_t rb = tile_id / n_tt, tt = tile_id % n_tt;
+    const int64_t sb0 = ks * a.ksb / splits, sb1 = (ks + 1) * a.ksb / splits;
+    const int64_t KSB = sb1 - sb0;                    // superblocks of this CTA
     const int64_t n_pieces = KSB * (256 / kPiece);
     unsigned* err = a.err;
 
@@ -148,7 +159,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
             mbar_init(c_full0 + 8 * i, 1);
             mbar_init(c_empty0 + 8 * i, kGemmDq);
         }
-        for (int i = 0; i < kXStages; i++) {
+        for (int i = 0; i < XS; i++) {
             mbar_init(x_full0 + 8 * i, 1);
             mbar_init(x_empty0 + 8 * i, 1);
         }
@@ -187,9 +198,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
                 mbar_arrive_expect_tx(fb, (uint32_t)(tiles * 512 * B + (kSigns ? 0 : 2 * kGScaleTile)));
                 for (int t = 0; t < tiles; t++)
                     tma_load_1d_hint(smem_u32(st + t * 512 * B),
-                                     a.packed + ((rb * 8 + t) * KSB + sb) * (int64_t)(512 * B), 512 * B, fb, pol);
+                                     a.packed + ((rb * 8 + t) * a.ksb + sb0 + sb) * (int64_t)(512 * B), 512 * B, fb,
+                                     pol);
                 if constexpr (!kSigns) {
-                    const int j0 = (int)((sb * 256) / GROUP) & ~7;
+                    const int j0 = (int)(((sb0 + sb) * 256) / GROUP) & ~7;
                     tma_load_2d(smem_u32(st + S.sc), &a.ms, j0, (int)(rb * 128), fb);
                     tma_load_2d(smem_u32(st + S.zr), &a.mz, j0, (int)(rb * 128), fb);
                 }
@@ -198,15 +210,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
     } else if (warp == kXWarp) {
         // ------------------------------------------------------------ activation producer
         if (lane == 0) {
-            for (int64_t p = 0; p < n_pieces && !*abort_flag; p++) {
-                const int xs = (int)(p % kXStages);
-                if (p >= kXStages && !mbar_wait_bounded(x_empty0 + 8 * xs, (uint32_t)(((p / kXStages) - 1) & 1), err)) {
+            // ring slot xs, and the parity of the slot's previous use (incremental, no divisions)
+            int xs = 0;
+            uint32_t xph = 1;
+            const int np = (int)n_pieces, pk0 = (int)(sb0 * 4);
+            for (int p = 0; p < np && !*abort_flag; p++) {
+                if (p >= XS && !mbar_wait_bounded(x_empty0 + 8 * xs, xph, err)) {
                     *abort_flag = 1;
                     break;
                 }
                 mbar_arrive_expect_tx(x_full0 + 8 * xs, (uint32_t)(NT * 128));
-                tma_load_2d(smem_u32(smem + S.x + xs * NT * 128), &a.mx, (int)(p * kPiece), (int)(tt * NT),
+                tma_load_2d(smem_u32(smem + S.x + xs * NT * 128), &a.mx, (pk0 + p) * kPiece, (int)(tt * NT),
                             x_full0 + 8 * xs);
+                if (++xs == XS) {
+                    xs = 0;
+                    xph ^= 1u;
+                }
             }
         }
     } else if (warp == 1) {
@@ -214,10 +233,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
         if (lane == 0) {
             // kind::f16 instruction descriptor: D fp32, A/B fp16, both K-major, N = NT, M = 128.
             constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-            for (int64_t p = 0; p < n_pieces; p++) {
-                const int as = (int)(p % kAStages), xs = (int)(p % kXStages);
-                if (*abort_flag || !mbar_wait_bounded(a_full0 + 8 * as, (uint32_t)((p / kAStages) & 1), err) ||
-                    !mbar_wait_bounded(x_full0 + 8 * xs, (uint32_t)((p / kXStages) & 1), err)) {
+            // ring slots and the parities to wait for (incremental: this thread is on the
+            // critical path once the tensor core is the bound)
+            int as = 0, xs = 0;
+            uint32_t aph = 0, xph = 0;
+            const int np = (int)n_pieces;
+            for (int p = 0; p < np; p++) {
+                if (*abort_flag || !mbar_wait_bounded(a_full0 + 8 * as, aph, err) ||
+                    !mbar_wait_bounded(x_full0 + 8 * xs, xph, err)) {
                     *abort_flag = 1;
                     break;
                 }
@@ -234,6 +257,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
                 }
                 umma_commit(a_empty0 + 8 * as);
                 umma_commit(x_empty0 + 8 * xs);
+                if (++as == kAStages) {
+                    as = 0;
+                    aph ^= 1u;
+                }
+                if (++xs == XS) {
+                    xs = 0;
+                    xph ^= 1u;
+                }
             }
             umma_commit(d_full);
             // All issued MMAs must finish before TMEM is freed, on the error path too.
@@ -284,8 +315,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
 #pragma unroll
                         for (int i = 0; i < 2; i++) {
                             const int kl = i ^ flip;            // 32-column block 2q + kl of the superblock
-                            *reinterpret_cast<uint4*>(abuf + a_sw128(row, 4 * kl + c)) =
-                                signs_octet(wa[u], wb[u], 2 * q + kl);
+                            sts128(smem_u32(abuf + a_sw128(row, 4 * kl + c)), signs_octet(wa[u], wb[u], 2 * q + kl));
                         }
                     }
                     fence_proxy_async_smem();
@@ -303,7 +333,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
             const uint8_t* tb = st + T * 512 * B + 16 * lane;
             const uint16_t* ss = reinterpret_cast<const uint16_t*>(st + S.sc);
             const uint16_t* zs = reinterpret_cast<const uint16_t*>(st + S.zr);
-            const int jbase = (int)((sb * 256) / GROUP) & ~7;
+            const int jbase = (int)(((sb0 + sb) * 256) / GROUP) & ~7;
             uint4 pl0 = make_uint4(0, 0, 0, 0), pl1 = make_uint4(0, 0, 0, 0);
             bool ok = true;
 #pragma unroll
@@ -323,7 +353,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
                 uint4 out[2][2];
 #pragma unroll
                 for (int kl = 0; kl < 2; kl++) {
-                    const int jj = (int)((sb * 256 + 64 * q + 32 * kl) / GROUP) - jbase;
+                    const int jj = (int)(((sb0 + sb) * 256 + 64 * q + 32 * kl) / GROUP) - jbase;
 #pragma unroll
                     for (int u = 0; u < 2; u++) {
                         const int row = 16 * T + g + 8 * u;
@@ -352,7 +382,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
                     for (int i = 0; i < 2; i++) {
                         const int kl = i ^ flip;
                         const uint4 v = flip ? out[u][i ^ 1] : out[u][i];
-                        *reinterpret_cast<uint4*>(abuf + a_sw128(row, 4 * kl + c)) = v;
+                        sts128(smem_u32(abuf + a_sw128(row, 4 * kl + c)), v);
                     }
                 }
                 fence_proxy_async_smem();
@@ -367,25 +397,82 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
             if (lane == 0) mbar_arrive(c_empty0 + 8 * cs);
         }
         // ------------------------------------------------------------ epilogue
-        if (mbar_wait_bounded(d_full, 0u, err, 1u << 26) && !*abort_flag) {
-            tc_fence_after();
-            const int quarter = warp & 3;                  // TMEM lanes this warp may access
-            const int half = (warp - 2) >> 2;              // which half of the NT columns
-            const int64_t row = rb * 128 + 32 * quarter + lane;
-            float rs = 1.0f;
-            if (a.rowscale != nullptr && row < a.n) rs = __half2float(__ushort_as_half(a.rowscale[row]));
+        // All eight warps take every named barrier (id 1) below, whatever happened before.
+        if (!mbar_wait_bounded(d_full, 0u, err, 1u << 26)) *abort_flag = 1;
+        named_barrier(1, kGemmDq * 32);
+        const bool ok = !*abort_flag;
+        tc_fence_after();
+        const int quarter = warp & 3;                  // TMEM lanes this warp may access
+        const int half = (warp - 2) >> 2;              // which half of the NT columns
+        const int rloc = 32 * quarter + lane;          // row inside the 128-row block
+        const int64_t row = rb * 128 + rloc;
+        float rs = 1.0f;
+        if (a.rowscale != nullptr && row < a.n) rs = __half2float(__ushort_as_half(a.rowscale[row]));
+        if (splits == 1) {
+            if (ok) {
 #pragma unroll 1
-            for (int c0 = half * (NT / 2); c0 < (half + 1) * (NT / 2); c0 += 16) {
-                uint32_t v[16];
-                tmem_ld16(tmem_d + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, v);
-                tmem_wait_ld();
-                if (row < a.n) {
+                for (int c0 = half * (NT / 2); c0 < (half + 1) * (NT / 2); c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem_d + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, v);
+                    tmem_wait_ld();
+                    if (row < a.n) {
 #pragma unroll
-                    for (int j = 0; j < 16; j++) {
-                        const int64_t tok = tt * NT + c0 + j;
-                        if (tok < a.M) a.y[tok * a.ldy + row] = from_f32<false>(__uint_as_float(v[j]) * rs);
+                        for (int j = 0; j < 16; j++) {
+                            const int64_t tok = tt * NT + c0 + j;
+                            if (tok < a.M) a.y[tok * a.ldy + row] = from_f32<false>(__uint_as_float(v[j]) * rs);
+                        }
                     }
                 }
+            }
+        } else {
+            // split-K: this slice's fp32 tile to its partial slot; the last slice to arrive
+            // (ticket) adds the slots in slice order and stores y (deterministic)
+            float* slot = a.partials + (tile_id * splits + ks) * (int64_t)(128 * NT);
+            if (ok) {
+#pragma unroll 1
+                for (int c0 = half * (NT / 2); c0 < (half + 1) * (NT / 2); c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem_d + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; j += 4)
+                        __stcg(reinterpret_cast<float4*>(slot + rloc * NT + c0 + j),
+                               make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                                           __uint_as_float(v[j + 3])));
+                }
+            }
+            __threadfence();
+            named_barrier(1, kGemmDq * 32);
+            if (threadIdx.x == kGemmDq0 * 32) {
+                // every slice takes its ticket, also after an error, so the counter returns to zero
+                const unsigned old = atomicAdd(a.counters + tile_id, 1u);
+                *last_flag = old == (unsigned)(splits - 1);
+            }
+            named_barrier(1, kGemmDq * 32);
+            if (*last_flag) {
+                __threadfence();
+                const float* p0 = a.partials + tile_id * splits * (int64_t)(128 * NT);
+                if (ok && row < a.n) {
+#pragma unroll 1
+                    for (int c0 = half * (NT / 2); c0 < (half + 1) * (NT / 2); c0 += 4) {
+                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int sl = 0; sl < splits; sl++) {
+                            const float4 t = __ldcg(reinterpret_cast<const float4*>(p0 + sl * (int64_t)(128 * NT) +
+                                                                                   rloc * NT + c0));
+                            acc.x += t.x;
+                            acc.y += t.y;
+                            acc.z += t.z;
+                            acc.w += t.w;
+                        }
+                        const float vv[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {
+                            const int64_t tok = tt * NT + c0 + j;
+                            if (tok < a.M) a.y[tok * a.ldy + row] = from_f32<false>(vv[j] * rs);
+                        }
+                    }
+                }
+                if (threadIdx.x == kGemmDq0 * 32) a.counters[tile_id] = 0u;
             }
         }
     }
@@ -456,16 +543,45 @@ static bool encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t co
 // Token tile: the smallest of 64 / 128 / 256 that holds M, 256 beyond.
 static int gemm_nt(int64_t M) { return M <= 64 ? 64 : (M <= 128 ? 128 : 256); }
 
+// Deepest activation ring (<= 8 stages) that fits the 227 KB of shared memory.
+static int gemm_xs(int B, int NT) {
+    int xs = kMaxXStages;
+    while (xs > 2 && GemmSmem(B, NT, xs).bytes + 1024 > 227 * 1024) xs--;
+    return xs;
+}
+
+// k slices per output tile.  Only grids smaller than one wave are split (each slice's fp32
+// partial tile is written and read back once, which larger grids cannot repay): as many
+// slices as keep the CTAs within one wave of the SMs, at most 8 and at least 4
+// superblocks a slice.
+static int gemm_splits(int64_t rows, int64_t M, int64_t ksb) {
+    const int64_t tiles = ceil_div(rows, (int64_t)128) * ceil_div(M, (int64_t)gemm_nt(M));
+    const int64_t sms = sm_count();
+    if (tiles >= sms) return 1;
+    int64_t s = sms / tiles;
+    s = std::min<int64_t>(s, 8);
+    s = std::min<int64_t>(s, std::max<int64_t>(1, ksb / 4));
+    return (int)std::max<int64_t>(1, s);
+}
+
+static size_t gemm_partials_bytes(int64_t rows, int64_t M, int64_t ksb) {
+    const int s = gemm_splits(rows, M, ksb);
+    if (s == 1) return 0;
+    const int64_t tiles = ceil_div(rows, (int64_t)128) * ceil_div(M, (int64_t)gemm_nt(M));
+    return (size_t)(tiles * s * 128 * gemm_nt(M) * 4);
+}
+
+// counter header | fp16 copy of bf16 activations | split-K partials
 size_t gemm_group_tc_ws_bytes(int64_t M, int64_t n, int64_t k) {
-    (void)n;
-    return kCounterBytes + (size_t)(M * k * 2 + 256);       // fp16 copy of bf16 activations
+    return kCounterBytes + al256((size_t)(M * k * 2)) + gemm_partials_bytes(n, M, k / 256);
 }
 
 bool gemm_group_tc_supported(int64_t M, int64_t n, int64_t k, int bits, int group) {
     if (M < 64 || n % 16 != 0 || k % 256 != 0 || bits < 2 || bits > 6) return false;
     if (group != 32 && group != 64 && group != 128) return false;
     if ((k / group) % 8 != 0 || M > ((int64_t)1 << 31) || n > ((int64_t)1 << 31)) return false;
-    return GemmSmem(bits, gemm_nt(M)).bytes + 1024 <= 227 * 1024;
+    if (ceil_div(n, (int64_t)128) * ceil_div(M, (int64_t)gemm_nt(M)) > kCounterBytes / 4) return false;
+    return GemmSmem(bits, gemm_nt(M), 2).bytes + 1024 <= 227 * 1024;
 }
 
 template <int B, int GROUP, int NT>
@@ -495,10 +611,12 @@ static lbq_status launch_gemm_g(int group, const GemmArgs& args, int64_t grid, s
 }
 
 template <int B>
-static lbq_status launch_gemm_b(int group, const GemmArgs& args, cudaStream_t st) {
+static lbq_status launch_gemm_b(int group, GemmArgs& args, cudaStream_t st) {
     const int NT = gemm_nt(args.M);
-    const int64_t grid = ceil_div(args.n, (int64_t)128) * ceil_div(args.M, (int64_t)NT);
-    const size_t smem = (size_t)GemmSmem(B, NT).bytes + 1024;   // + room to align the base to 1024
+    args.xs = gemm_xs(B, NT);
+    args.splits = gemm_splits(args.n, args.M, args.ksb);
+    const int64_t grid = ceil_div(args.n, (int64_t)128) * ceil_div(args.M, (int64_t)NT) * args.splits;
+    const size_t smem = (size_t)GemmSmem(B, NT, args.xs).bytes + 1024;   // + room to align the base to 1024
     if (NT == 64) return launch_gemm_g<B, 64>(group, args, grid, smem, st);
     if (NT == 128) return launch_gemm_g<B, 128>(group, args, grid, smem, st);
     return launch_gemm_g<B, 256>(group, args, grid, smem, st);
@@ -530,6 +648,8 @@ lbq_status launch_gemm_group_tc(const void* x, bool bf16, int64_t M, const void*
     args.M = M;
     args.ldy = n;
     args.err = device_error_word();
+    args.counters = (unsigned*)ws;
+    args.partials = (float*)((char*)ws + kCounterBytes + al256((size_t)(M * k * 2)));
     switch (bits) {
         case 2: return launch_gemm_b<2>(group, args, st);
         case 3: return launch_gemm_b<3>(group, args, st);
@@ -550,29 +670,35 @@ lbq_status launch_gemm_group_tc(const void* x, bool bf16, int64_t M, const void*
 struct BinGemmWs {
     uint16_t* xs;      // fp16(s2 . x) [M x d_in]
     uint16_t* t;       // fp16 [M x ldt]
+    float* partials;   // split-K partial tiles
     int64_t ldt;
     size_t bytes;
 };
 
-static BinGemmWs bin_gemm_ws(void* base, int64_t M, int64_t d_in, int64_t r) {
+static BinGemmWs bin_gemm_ws(void* base, int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
     BinGemmWs w{};
-    const size_t xs_bytes = ((size_t)(M * d_in * 2) + 255) / 256 * 256;
+    const size_t xs_bytes = al256((size_t)(M * d_in * 2));
     w.ldt = sign_cols_pad(r);
     w.xs = (uint16_t*)((char*)base + kCounterBytes);
     w.t = (uint16_t*)((char*)base + kCounterBytes + xs_bytes);
-    w.bytes = kCounterBytes + xs_bytes + (size_t)(M * w.ldt * 2);
+    const size_t t_bytes = al256((size_t)(M * w.ldt * 2));
+    w.partials = (float*)((char*)base + kCounterBytes + xs_bytes + t_bytes);
+    // the stages run one after the other and share the partials region
+    w.bytes = kCounterBytes + xs_bytes + t_bytes +
+              std::max(gemm_partials_bytes(r, M, sign_cols_pad(d_in) / 256),
+                       gemm_partials_bytes(d_out, M, sign_cols_pad(r) / 256));
     return w;
 }
 
 size_t gemm_binlr_tc_ws_bytes(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
-    (void)d_out;
-    return bin_gemm_ws(nullptr, M, d_in, r).bytes;
+    return bin_gemm_ws(nullptr, M, d_out, d_in, r).bytes;
 }
 
 bool gemm_binlr_tc_supported(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
     if (M < 64 || d_out % 16 != 0 || r % 32 != 0 || d_in % 32 != 0) return false;
     if (M > ((int64_t)1 << 31) || d_out > ((int64_t)1 << 31) || r > ((int64_t)1 << 31)) return false;
-    return GemmSmem(1, gemm_nt(M)).bytes + 1024 <= 227 * 1024;
+    if (ceil_div(std::max(d_out, r), (int64_t)128) * ceil_div(M, (int64_t)gemm_nt(M)) > kCounterBytes / 4) return false;
+    return GemmSmem(1, gemm_nt(M), 2).bytes + 1024 <= 227 * 1024;
 }
 
 lbq_status launch_gemm_binlr_tc(const void* x, bool bf16, int64_t M, const void* U, const void* Vt, const void* s1,
@@ -580,7 +706,7 @@ lbq_status launch_gemm_binlr_tc(const void* x, bool bf16, int64_t M, const void*
                                 size_t ws_bytes, cudaStream_t st) {
     if (ws == nullptr || ws_bytes < gemm_binlr_tc_ws_bytes(M, d_out, d_in, r)) return LBQ_ERR_WORKSPACE;
     if (gemm_encode_fn() == nullptr) return LBQ_ERR_CUDA;
-    const BinGemmWs w = bin_gemm_ws(ws, M, d_in, r);
+    const BinGemmWs w = bin_gemm_ws(ws, M, d_out, d_in, r);
     lbq_status s = to_f16(x, bf16, s2, M, d_in, w.xs, st);
     if (s != LBQ_OK) return s;
     const int NT = gemm_nt(M);
@@ -595,6 +721,8 @@ lbq_status launch_gemm_binlr_tc(const void* x, bool bf16, int64_t M, const void*
     a1.M = M;
     a1.ldy = w.ldt;
     a1.err = device_error_word();
+    a1.counters = (unsigned*)ws;
+    a1.partials = w.partials;
     s = launch_gemm_b<1>(32, a1, st);
     if (s != LBQ_OK) return s;
     GemmArgs a2;
@@ -608,6 +736,8 @@ lbq_status launch_gemm_binlr_tc(const void* x, bool bf16, int64_t M, const void*
     a2.M = M;
     a2.ldy = d_out;
     a2.err = a1.err;
+    a2.counters = (unsigned*)ws;
+    a2.partials = w.partials;
     return launch_gemm_b<1>(32, a2, st);
 }
 

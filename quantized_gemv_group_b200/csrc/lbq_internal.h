@@ -31,6 +31,8 @@ struct GroupGeom {
 inline int64_t group_superblock(int bits) { return (bits >= 2 && bits <= 6) ? 256 : 0; }
 
 inline int64_t sign_cols_pad(int64_t cols) { return (cols + 255) / 256 * 256; }
+inline size_t al256(size_t v) { return (v + 255) / 256 * 256; }
+inline int al16(int64_t v) { return (int)((v + 15) / 16 * 16); }
 
 // Every workspace starts with a fixed header of ticket counters (one per 16-row
 // tile, at most kMaxTiles).  It must be zero before the first call; every call

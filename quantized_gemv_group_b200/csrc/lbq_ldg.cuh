@@ -95,8 +95,6 @@ __device__ __forceinline__ PrepOut prep_quantize8(const float (&v)[8], int E) {
 }
 
 // ------------------------------------------------------------------ host side
-inline size_t al256(size_t v) { return (v + 255) / 256 * 256; }
-inline int al16(int64_t v) { return (int)((v + 15) / 16 * 16); }
 
 template <class Kern, class... Args>
 inline lbq_status launch_pdl(Kern kern, int grid, int threads, size_t smem, cudaStream_t st, const Args&... args) {

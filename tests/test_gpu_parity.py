@@ -252,6 +252,33 @@ def test_gemm_group_tc_sweep(bits, group, M):
     assert np.max(np.abs(yf - ref)) <= 2e-2 * scale
 
 
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 32), (6, 64)])
+@pytest.mark.parametrize("M", [64, 200])
+def test_gemm_group_tc_split_k(bits, group, M):
+    # 2 row blocks with k = 4096 (16 superblocks): the tile count is far below the SM count,
+    # so k is split in 4 slices whose fp32 partials are added by the last slice to finish
+    n, k = 256, 4096
+    W, x, codes, s, z = _group_case(n, k, bits, group, M, seed=11 * bits + M, xdtype=torch.bfloat16)
+    ref = _oracle_group(x, codes, s, z, n, k, bits, group)
+    packed = lbq.lbq_pack(codes, bits)
+    y1 = lbq.lbq_gemm_group(x, packed, s, z, n, k, bits, group).clone()
+    y2 = lbq.lbq_gemm_group(x, packed, s, z, n, k, bits, group).clone()
+    torch.cuda.synchronize()
+    assert lbq.lbq_last_device_error() == 0
+    assert _rel(_np(y1.float()), ref) <= REL_TOL
+    assert torch.equal(y1, y2)                     # fixed slice order: deterministic
+
+
+def test_gemm_binlr_tc_split_k():
+    d_out, d_in, r, M = 256, 4096, 64, 100
+    Uw, Vw, s1, s2, x = _binlr_case(d_out, d_in, r, M, seed=77)
+    y = _binlr_run(Uw, Vw, s1, s2, x, d_out, d_in, r, lbq.LAYOUT_KERNEL, fn=lbq.lbq_gemm_binlr)
+    torch.cuda.synchronize()
+    assert lbq.lbq_last_device_error() == 0
+    ref = _binlr_oracle(Uw, Vw, s1, s2, x, d_out, d_in, r)
+    assert _rel(_np(y.float()), ref) <= REL_TOL
+
+
 def test_gemm_group_tc_deterministic_and_matches_gemv_blocks():
     n, k, M = 256, 2048, 96
     W, x, codes, s, z = _group_case(n, k, 4, 64, M, seed=31)
