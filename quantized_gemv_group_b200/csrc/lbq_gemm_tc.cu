@@ -8,14 +8,14 @@
 // and the product becomes a dense contraction worth the 5th-generation tensor cores.
 // One CTA computes a 128-row x NT-token tile of y^T in tensor memory (TMEM):
 //
-//  * warp 0 streams, with the Tensor Memory Accelerator (TMA), the packed codes of the
-//    eight 16-row tiles for one 256-wide k superblock plus the 128 x 8 scale and zero
-//    boxes into a ring of code stages;
+//  * warps 2..9 (one per 16-row tile) each stream their tile's packed codes and its 16 x 8
+//    scale and zero boxes, superblock by superblock, into a ring of their own with cp.async
+//    (one 16-byte piece per lane and 512-byte block: the bulk-copy engine's throughput per
+//    CTA follows the number of copies, plain async loads do not), expand them to fp16
+//    weights w = fp16(s * (q - z)) for the 128 x 64 A piece, K-major with 128-byte swizzle,
+//    and at the end read the fp32 accumulator back from TMEM and store y in fp16;
 //  * warp 10 streams the activations x (fp16) in 64-wide k pieces through a 2-D tensor
-//    map with 128-byte swizzle, the K-major layout the tensor core reads;
-//  * warps 2..9 (one per 16-row tile) expand the codes to fp16 weights
-//    w = fp16(s * (q - z)) for the 128 x 64 A piece, K-major with 128-byte swizzle; at
-//    the end they read the fp32 accumulator back from TMEM and store y in fp16;
+//    map (TMA) with 128-byte swizzle, the K-major layout the tensor core reads;
 //  * warp 1 allocates TMEM and one of its threads issues tcgen05.mma.kind::f16
 //    (M = 128, N = NT, K = 16) from shared-memory descriptors; tcgen05.commit frees the
 //    A and x buffers and finally signals the epilogue.
@@ -35,31 +35,32 @@ constexpr int kGemmDq0 = 2;                        // first dequant warp
 constexpr int kGemmThreads = (3 + kGemmDq) * 32;   // codes producer, MMA, dequant x8, x producer
 constexpr int kXWarp = 2 + kGemmDq;
 constexpr int kPiece = 64;                         // k per A piece = one 128-byte swizzle row
-constexpr int kCodeStages = 3;
+constexpr int kWarpRing = 3;                       // superblocks in flight per dequant warp
 constexpr int kMaxXStages = 8;                     // activation ring depth: as deep as shared memory allows
-constexpr int kAStages = 2;
+constexpr int kAStages = 4;                        // A pieces between dequant and tensor core
 constexpr int kGScaleBox = 8;                      // groups per scale/zero box
-constexpr int kGScaleTile = 128 * kGScaleBox * 2;  // bytes of one 128 x 8 fp16 box
 constexpr int kAStageBytes = 128 * kPiece * 2;     // 16 KB
 
 // B = 2..6: group codes with scale/zero boxes; B = 1: a +-1 sign matrix (no scales).
+// Each dequant warp owns a ring of kWarpRing slots: its tile's 512 * B bytes of one
+// superblock, then (group codes) the tile's 16 rows x 8 groups of scales and of zeros.
 struct GemmSmem {
-    int x, a, codes, code_stage, sc, zr, bars, bytes;
+    int x, a, codes, slot, bars, bytes;
     __host__ __device__ GemmSmem(int B, int NT, int XS) {
         x = 0;                                           // every stage 1024-byte aligned
         a = x + XS * NT * 128;
         codes = a + kAStages * kAStageBytes;
-        code_stage = 4096 * B + (B > 1 ? 2 * kGScaleTile : 0);
-        sc = 4096 * B;                                   // offsets inside a code stage
-        zr = sc + kGScaleTile;
-        bars = codes + kCodeStages * code_stage;
-        bytes = bars + 256;
+        slot = 512 * B + (B > 1 ? 2 * 16 * kGScaleBox * 2 : 0);
+        bars = codes + kGemmDq * kWarpRing * slot;
+        bytes = bars + 512;
     }
 };
 
 struct GemmArgs {
     CUtensorMap mx;        // B operand (fp16) [M x k], box 64 x NT, 128-byte swizzle
-    CUtensorMap ms, mz;    // scales / zeros [n x k/g] fp16, box 8 x 128 (group codes only)
+    const uint16_t* scales;    // group codes: [n x ngroups] fp16 scales and zeros
+    const uint16_t* zeros;
+    int64_t ngroups;
     const uint8_t* packed; // A in its kernel layout: 16-row tiles x 256-wide k superblocks
     const uint16_t* rowscale;  // optional fp16 factor per output row (signs: s1), else null
     uint16_t* y;           // fp16 [M x ldy]
@@ -133,15 +134,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
     const int XS = a.xs;
     const GemmSmem S(B, NT, XS);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S.bars);
-    // c_full[3] c_empty[3] x_full[8] x_empty[8] a_full[2] a_empty[2] d_full | tmem address |
-    // abort flag | split ticket result
-    const uint32_t c_full0 = smem_u32(&bars[0]), c_empty0 = smem_u32(&bars[3]);
-    const uint32_t x_full0 = smem_u32(&bars[6]), x_empty0 = smem_u32(&bars[6 + kMaxXStages]);
-    const uint32_t a_full0 = smem_u32(&bars[6 + 2 * kMaxXStages]), a_empty0 = smem_u32(&bars[8 + 2 * kMaxXStages]);
-    const uint32_t d_full = smem_u32(&bars[10 + 2 * kMaxXStages]);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[11 + 2 * kMaxXStages]);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[12 + 2 * kMaxXStages]);
-    volatile int* last_flag = reinterpret_cast<volatile int*>(&bars[13 + 2 * kMaxXStages]);
+    // x_full[8] x_empty[8] a_full[4] a_empty[4] d_full | tmem address | abort flag | split
+    // ticket result
+    constexpr int kXb = kMaxXStages, kAb = kAStages;
+    const uint32_t x_full0 = smem_u32(&bars[0]), x_empty0 = smem_u32(&bars[kXb]);
+    const uint32_t a_full0 = smem_u32(&bars[2 * kXb]), a_empty0 = smem_u32(&bars[2 * kXb + kAb]);
+    const uint32_t d_full = smem_u32(&bars[2 * kXb + 2 * kAb]);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2 * kXb + 2 * kAb + 1]);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[2 * kXb + 2 * kAb + 2]);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(&bars[2 * kXb + 2 * kAb + 3]);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n_tt = (a.M + NT - 1) / NT;
@@ -155,10 +156,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
     unsigned* err = a.err;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kCodeStages; i++) {
-            mbar_init(c_full0 + 8 * i, 1);
-            mbar_init(c_empty0 + 8 * i, kGemmDq);
-        }
         for (int i = 0; i < XS; i++) {
             mbar_init(x_full0 + 8 * i, 1);
             mbar_init(x_empty0 + 8 * i, 1);
@@ -181,32 +178,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
     const uint32_t tmem_d = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ codes + scales producer
-        if (lane == 0) {
-            const uint64_t pol = l2_policy_evict_first();
-            const int64_t tiles_left = a.n / 16 - rb * 8;
-            const int tiles = (int)(tiles_left < 8 ? tiles_left : 8);
-            for (int64_t sb = 0; sb < KSB && !*abort_flag; sb++) {
-                const int s = (int)(sb % kCodeStages);
-                if (sb >= kCodeStages &&
-                    !mbar_wait_bounded(c_empty0 + 8 * s, (uint32_t)(((sb / kCodeStages) - 1) & 1), err)) {
-                    *abort_flag = 1;
-                    break;
-                }
-                uint8_t* st = smem + S.codes + s * S.code_stage;
-                const uint32_t fb = c_full0 + 8 * s;
-                mbar_arrive_expect_tx(fb, (uint32_t)(tiles * 512 * B + (kSigns ? 0 : 2 * kGScaleTile)));
-                for (int t = 0; t < tiles; t++)
-                    tma_load_1d_hint(smem_u32(st + t * 512 * B),
-                                     a.packed + ((rb * 8 + t) * a.ksb + sb0 + sb) * (int64_t)(512 * B), 512 * B, fb,
-                                     pol);
-                if constexpr (!kSigns) {
-                    const int j0 = (int)(((sb0 + sb) * 256) / GROUP) & ~7;
-                    tma_load_2d(smem_u32(st + S.sc), &a.ms, j0, (int)(rb * 128), fb);
-                    tma_load_2d(smem_u32(st + S.zr), &a.mz, j0, (int)(rb * 128), fb);
-                }
-            }
-        }
+        // (idle: the dequant warps fetch their own codes, scales and zeros)
     } else if (warp == kXWarp) {
         // ------------------------------------------------------------ activation producer
         if (lane == 0) {
@@ -278,19 +250,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
         const int flip = g & 1;                         // store order that keeps 8-lane phases conflict-free
         constexpr int O0 = 4 / W0;
         constexpr int O1 = W1 > 0 ? 4 / W1 : 1;
-        for (int64_t sb = 0; sb < KSB && !*abort_flag; sb++) {
-            const int cs = (int)(sb % kCodeStages);
-            if (!mbar_wait_bounded(c_full0 + 8 * cs, (uint32_t)((sb / kCodeStages) & 1), err)) {
-                *abort_flag = 1;
-                break;
+        // This warp's ring: cp.async of its tile's superblock (one 16-byte piece per lane per
+        // 512-byte plane block) and of 16 rows x 8 groups of scales and zeros (lane i: row
+        // i mod 16 of the scales, i < 16, or of the zeros), kWarpRing superblocks ahead.
+        uint8_t* cring = smem + S.codes + T * kWarpRing * S.slot;
+        const bool tile_live = rb * 8 + T < a.n / 16;
+        auto issue_ring = [&](int slot, int64_t sb) {
+            if (!tile_live) return;
+            uint8_t* dst = cring + slot * S.slot;
+            const uint8_t* src = a.packed + ((rb * 8 + T) * a.ksb + sb0 + sb) * (int64_t)(512 * B) + 16 * lane;
+#pragma unroll
+            for (int i = 0; i < B; i++) cp_async_cg16(smem_u32(dst + 512 * i + 16 * lane), src + 512 * i);
+            if constexpr (!kSigns) {
+                const int r = lane & 15, arr = lane >> 4;
+                const int64_t j0 = (((sb0 + sb) * 256) / GROUP) & ~(int64_t)7;
+                const uint16_t* sp = (arr ? a.zeros : a.scales) + (rb * 128 + 16 * T + r) * a.ngroups + j0;
+                cp_async_cg16(smem_u32(dst + 512 * B + arr * (16 * kGScaleBox * 2) + r * (kGScaleBox * 2)), sp);
             }
-            const uint8_t* st = smem + S.codes + cs * S.code_stage;
+        };
+#pragma unroll 1
+        for (int i = 0; i < kWarpRing; i++) {
+            if (i < KSB) issue_ring(i, i);
+            cp_async_commit();
+        }
+        int ring_slot = 0;
+        for (int64_t sb = 0; sb < KSB && !*abort_flag; sb++) {
+            cp_async_wait<kWarpRing - 1>();
+            __syncwarp();
+            const uint8_t* st = cring + ring_slot * S.slot;
             if constexpr (kSigns) {
                 // Sign layout: lane L = 4g + c holds words (row g, cols 4c..4c+3 of each
                 // 32-column block p at bit 8j + p), (row g+8, same), (row g, cols 16 + ...),
                 // (row g+8, cols 16 + ...).  The octet 8c..8c+7 of a block comes from lanes
                 // 4g + 2(c mod 2) and 4g + 2(c mod 2) + 1, word u + 2(c / 2).
-                const uint32_t* tw = reinterpret_cast<const uint32_t*>(st + T * 512);
+                const uint32_t* tw = reinterpret_cast<const uint32_t*>(st);
                 const int la = 4 * g + 2 * (c & 1);
                 uint32_t wa[2], wb[2];
 #pragma unroll
@@ -327,12 +320,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
                     break;
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(c_empty0 + 8 * cs);
+                if (sb + kWarpRing < KSB) issue_ring(ring_slot, sb + kWarpRing);
+                cp_async_commit();
+                ring_slot = ring_slot + 1 == kWarpRing ? 0 : ring_slot + 1;
                 continue;
             }
-            const uint8_t* tb = st + T * 512 * B + 16 * lane;
-            const uint16_t* ss = reinterpret_cast<const uint16_t*>(st + S.sc);
-            const uint16_t* zs = reinterpret_cast<const uint16_t*>(st + S.zr);
+            const uint8_t* tb = st + 16 * lane;
+            const uint16_t* ss = reinterpret_cast<const uint16_t*>(st + 512 * B);   // [16 rows][8 groups]
+            const uint16_t* zs = ss + 16 * kGScaleBox;
             const int jbase = (int)(((sb0 + sb) * 256) / GROUP) & ~7;
             uint4 pl0 = make_uint4(0, 0, 0, 0), pl1 = make_uint4(0, 0, 0, 0);
             bool ok = true;
@@ -356,7 +351,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
                     const int jj = (int)(((sb0 + sb) * 256 + 64 * q + 32 * kl) / GROUP) - jbase;
 #pragma unroll
                     for (int u = 0; u < 2; u++) {
-                        const int row = 16 * T + g + 8 * u;
                         const int eta = 4 * q + 2 * kl + u;
                         const int wi0 = (eta / O0) & 3, o0 = eta % O0;
                         const uint32_t* p0 = &pl0.x;
@@ -368,8 +362,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
                             w1 = p1[(eta / O1) & 3];
                             o1 = eta % O1;
                         }
-                        const uint16_t sh = ss[row * kGScaleBox + jj];
-                        const __half zh = __hadd(__ushort_as_half(zs[row * kGScaleBox + jj]), __float2half(1024.f));
+                        const int lrow = g + 8 * u;                   // row inside the warp's tile
+                        const uint16_t sh = ss[lrow * kGScaleBox + jj];
+                        const __half zh = __hadd(__ushort_as_half(zs[lrow * kGScaleBox + jj]), __float2half(1024.f));
                         const uint32_t zz2 = (uint32_t)__half_as_ushort(zh) * 0x00010001u;
                         const uint32_t ss2 = (uint32_t)sh * 0x00010001u;
                         out[u][kl] = dequant_octet<W0, W1>(w0, w1, o0, o1, zz2, ss2);
@@ -394,8 +389,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_group_tc05(const __gri
                 break;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(c_empty0 + 8 * cs);
+            if (sb + kWarpRing < KSB) issue_ring(ring_slot, sb + kWarpRing);
+            cp_async_commit();
+            ring_slot = ring_slot + 1 == kWarpRing ? 0 : ring_slot + 1;
         }
+        cp_async_wait<0>();
         // ------------------------------------------------------------ epilogue
         // All eight warps take every named barrier (id 1) below, whatever happened before.
         if (!mbar_wait_bounded(d_full, 0u, err, 1u << 26)) *abort_flag = 1;
@@ -636,10 +634,10 @@ lbq_status launch_gemm_group_tc(const void* x, bool bf16, int64_t M, const void*
     }
     GemmArgs args;
     memset(&args, 0, sizeof args);
-    if (!encode_2d(&args.mx, xf, M, k, k, 64, (uint32_t)gemm_nt(M), CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&args.ms, scales, n, k / group, k / group, kGScaleBox, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_2d(&args.mz, zeros, n, k / group, k / group, kGScaleBox, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return LBQ_ERR_CUDA;
+    if (!encode_2d(&args.mx, xf, M, k, k, 64, (uint32_t)gemm_nt(M), CU_TENSOR_MAP_SWIZZLE_128B)) return LBQ_ERR_CUDA;
+    args.scales = (const uint16_t*)scales;
+    args.zeros = (const uint16_t*)zeros;
+    args.ngroups = k / group;
     args.packed = (const uint8_t*)packed;
     args.rowscale = nullptr;
     args.y = (uint16_t*)y;
