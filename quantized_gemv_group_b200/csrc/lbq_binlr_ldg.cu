@@ -8,17 +8,16 @@
 //   stage 2: y[m, i] = s1[i] * sum_j U[i, j] * t[m, j]         rows d_out, columns r
 //
 //  * Every CTA prepares the stage input v (s2 . x, or t) in its shared memory right after
-//    waiting for the previous kernel: one power-of-two scale 2^E per token over the whole
-//    vector (|v| <= 32639 after scaling), int8 planes hi, lo (v = 256 hi + lo) in
-//    B-fragment order and exact per-256-chunk sums of v.
+//    waiting for the previous kernel, in one pass: one power-of-two scale 2^E per token and
+//    256-column chunk (|v| <= 32639 after scaling), int8 planes hi, lo (v = 256 hi + lo) in
+//    B-fragment order and the exact chunk sums of v.
 //  * Warps split the (16-row tile, 256-column superblock) units evenly (warp-level
 //    stream-K) and stream the lanes' 16-byte sign words straight into registers, several
-//    units ahead.  Per k-step a word masked with 0x01010101 << p gives four u8 A-fragment
-//    bytes 2^p * bit (one LOP per four signs); mma.m16n8k32 u8 x s8 accumulates each p in
-//    its own set, and at the tile's end S = sum_p acc_p >> p = sum bit * v exactly.
-//  * sum_k sign * v = 2 S - sum v; the partial of a warp is 2^E (2 S - sum of v over its
-//    superblocks) (times s1 in stage 2); tiles split between warps are finished in fixed
-//    order by the last one to arrive (tile_epilogue), so the result is deterministic.
+//    units ahead.  Per k-step p the word's bits p of each byte give four 0/1 u8 A-fragment
+//    bytes; mma.m16n8k32 u8 x s8 gives S = sum bit * v over the unit exactly.
+//  * sum_k sign * v = 2 S - sum v; each unit adds 2^E (2 S - chunk sum) to the warp's fp32
+//    partial (times s1 in stage 2); tiles split between warps are finished in fixed order
+//    by the last one to arrive (tile_epilogue), so the result is deterministic.
 //  * Both launches are programmatic dependents; only their first weight loads precede the
 //    wait for the previous kernel.
 #include <cstring>
@@ -143,37 +142,22 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_binlr_ldg(const __grid_const
     lptr += D * 512;
     if (lane < PF && u_begin + D + lane < u_end) l2_prefetch_bulk(lptr - 16 * lane + lane * 512, 512);
     if (threadIdx.x < 16) reinterpret_cast<uint4*>(smem + a.szero)[threadIdx.x] = make_uint4(0, 0, 0, 0);
-    int* maxbits = reinterpret_cast<int*>(smem + a.se) + 4;      // |v| maxima (float bits), M <= 4
-    if (threadIdx.x < 4) maxbits[threadIdx.x] = 0;
     griddep_wait();
-    __syncthreads();
 
-    // ---- prepare the stage input: per-token maxima, then planes and chunk sums; the chunk
-    // order is rotated by the CTA index so that the CTAs do not all read the same lines
+    // ---- prepare the stage input in one pass: per 256-column chunk one power-of-two scale,
+    // the int8 planes and the exact chunk sum; the chunk order is rotated by the CTA index
+    // so that the CTAs do not all read the same lines at once
     const int kch = (int)(a.cpad / kLdgChunk);
     const int rot = (int)(blockIdx.x % (unsigned)kch);
-    for (int m = 0; m < M; m++) {
-        float mx = 0.0f;
-        for (int cw = warp; cw < kch; cw += kBinWarpsPerCta) {
-            const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
-            float v[8];
-            bin_load8<STAGE2, BF16>(a, m, (int64_t)ch * kLdgChunk + 8 * lane, v);
-            mx = fmaxf(mx, warp_max_abs8(v));
-        }
-        if (lane == 0) atomicMax(&maxbits[m], __float_as_int(mx));   // non-negative floats order as ints
-    }
-    __syncthreads();
     int* expo = reinterpret_cast<int*>(smem + a.se);
     int* vsum = reinterpret_cast<int*>(smem + a.sv);
     for (int m = 0; m < M; m++) {
-        const int E = ldg_fixed_point_exponent(__int_as_float(maxbits[m]));
-        if (threadIdx.x == 0) expo[m] = E;
         int8_t* row_h = reinterpret_cast<int8_t*>(smem + a.sp) + (int64_t)(2 * m) * a.cpad;
         for (int cw = warp; cw < kch; cw += kBinWarpsPerCta) {
             const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
             float v[8];
             bin_load8<STAGE2, BF16>(a, m, (int64_t)ch * kLdgChunk + 8 * lane, v);
-            const PrepOut r = bin_quantize8(v, E);
+            const PrepOut r = bin_quantize8(v, ldg_fixed_point_exponent(warp_max_abs8(v)));
             // elements 8 lane + 0..3 and + 4..7: columns 32p + 16h + 4c' + j
             const int p = lane >> 2, h = (lane & 3) >> 1, c0 = 2 * (lane & 1);
             int8_t* base = row_h + ch * kLdgChunk;
@@ -181,7 +165,10 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_binlr_ldg(const __grid_const
             *reinterpret_cast<uint32_t*>(base + bin_plane_off(p, h, c0 + 1)) = r.hi.y;
             *reinterpret_cast<uint32_t*>(base + a.cpad + bin_plane_off(p, h, c0)) = r.lo.x;
             *reinterpret_cast<uint32_t*>(base + a.cpad + bin_plane_off(p, h, c0 + 1)) = r.lo.y;
-            if (lane == 0) vsum[m * kch + ch] = r.gsum;
+            if (lane == 0) {
+                vsum[m * kch + ch] = r.gsum;
+                expo[m * kch + ch] = r.E;
+            }
         }
     }
     __syncthreads();
@@ -194,15 +181,10 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_binlr_ldg(const __grid_const
     const int pstep = pv ? kLdgChunk : 0;
     const bool tv = c < M;
     const int* vrow = tv ? vsum + c * kch : reinterpret_cast<const int*>(smem + a.szero);
+    const int* erow = tv ? expo + c * kch : reinterpret_cast<const int*>(smem + a.szero);
     const int vstep = tv ? 1 : 0;
-    const float scale = tv ? ldg_exp2i(expo[c]) : 0.0f;
 
-    int acc[8][4];
-#pragma unroll
-    for (int p = 0; p < 8; p++)
-#pragma unroll
-        for (int e = 0; e < 4; e++) acc[p][e] = 0;
-    int vpart = 0;                                   // sum of v over this warp's superblocks of the tile
+    float part0 = 0.0f, part1 = 0.0f;                // rows g and g + 8 of token c, this warp's slice
     int tile_first_u = u_begin - csb;
 
     for (int base = u_begin; base < u_end; base += D) {
@@ -216,30 +198,29 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_binlr_ldg(const __grid_const
                     lptr += 512;
                 }
                 const int8_t* pr = prow + csb * pstep;
+                // S = sum over the unit of bit * v, exactly: 0/1 A bytes of k-step p
+                int s[4];
 #pragma unroll
                 for (int p = 0; p < 8; p += 2) {
                     const uint4 bq = *reinterpret_cast<const uint4*>(pr + 64 * (p >> 1));
 #pragma unroll
                     for (int q = 0; q < 2; q++) {
-                        const uint32_t msk = 0x01010101u << (p + q);
-                        mma_16832_u8s8(acc[p + q], w.x & msk, w.y & msk, w.z & msk, w.w & msk, q ? bq.z : bq.x,
-                                       q ? bq.w : bq.y);
+                        const int sh = p + q;
+                        const uint32_t a0 = (w.x >> sh) & 0x01010101u, a1 = (w.y >> sh) & 0x01010101u;
+                        const uint32_t a2 = (w.z >> sh) & 0x01010101u, a3 = (w.w >> sh) & 0x01010101u;
+                        if (sh == 0) mma_16832_u8s8_zc(s, a0, a1, a2, a3, bq.x, bq.y);
+                        else mma_16832_u8s8(s, a0, a1, a2, a3, q ? bq.z : bq.x, q ? bq.w : bq.y);
                     }
                 }
-                vpart += vrow[csb * vstep];
+                // sum_k sign * v = 2 S - sum v, times this chunk's 2^E; columns 2c (hi), 2c + 1 (lo)
+                const int vs = vrow[csb * vstep];
+                const float sc = ldg_exp2i(erow[csb * vstep]);
+                part0 = fmaf(sc, (float)(2 * (256 * s[0] + s[1]) - vs), part0);
+                part1 = fmaf(sc, (float)(2 * (256 * s[2] + s[3]) - vs), part1);
                 if (csb == ksb - 1 || u == u_end - 1) {
-                    // S = sum_p acc_p >> p; columns 2c (hi) and 2c + 1 (lo) of token c
-                    int s[4];
-#pragma unroll
-                    for (int e = 0; e < 4; e++) {
-                        int v = 0;
-#pragma unroll
-                        for (int p = 0; p < 8; p++) v += acc[p][e] >> p;
-                        s[e] = v;
-                    }
                     float part[NB][2];
-                    part[0][0] = scale * (float)(2 * (256 * s[0] + s[1]) - vpart);
-                    part[0][1] = scale * (float)(2 * (256 * s[2] + s[3]) - vpart);
+                    part[0][0] = tv ? part0 : 0.0f;
+                    part[0][1] = tv ? part1 : 0.0f;
                     const int64_t row = (int64_t)ct * 16 + g;
                     if constexpr (STAGE2) {
                         part[0][0] *= __half2float(__ushort_as_half(a.s1[row]));
@@ -252,11 +233,7 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_binlr_ldg(const __grid_const
                     else
                         tile_epilogue_f32<NB>(part, full, M, a.rows, ct, ct, (int64_t)ct * ksb, ksb, S, W, wid,
                                               a.partials, a.counters, a.maxc, a.tout);
-#pragma unroll
-                    for (int p = 0; p < 8; p++)
-#pragma unroll
-                        for (int e = 0; e < 4; e++) acc[p][e] = 0;
-                    vpart = 0;
+                    part0 = part1 = 0.0f;
                     tile_first_u = u + 1;
                 }
                 if (++csb == ksb) {
@@ -296,8 +273,8 @@ static BinLdgPlan bin_ldg_plan(int64_t M, int64_t d_out, int64_t d_in, int64_t r
 }
 
 static int bin_smem_bytes(int64_t M, int64_t cpad) {
-    // planes [2M][cpad] | chunk sums [M][cpad/256] | exponents and maxima (8 ints) | zero chunk
-    return al16(2 * M * cpad) + al16(M * (cpad / kLdgChunk) * 4) + 32 + 256;
+    // planes [2M][cpad] | chunk sums [M][cpad/256] | chunk exponents [M][cpad/256] | zero chunk
+    return al16(2 * M * cpad) + 2 * al16(M * (cpad / kLdgChunk) * 4) + 256;
 }
 
 bool gemv_binlr_ldg_supported(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
@@ -354,7 +331,7 @@ lbq_status launch_gemv_binlr_ldg(const void* x, bool bf16, int64_t M, const void
         a.sp = 0;
         a.sv = al16(2 * M * a.cpad);
         a.se = a.sv + al16(M * a.ksb * 4);
-        a.szero = a.se + 32;
+        a.szero = a.se + al16(M * a.ksb * 4);
         const int smem = bin_smem_bytes(M, a.cpad);
         const int grid = st2 ? pl.grid2 : pl.grid1;
         lbq_status s;
