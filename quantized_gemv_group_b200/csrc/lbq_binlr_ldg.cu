@@ -16,11 +16,13 @@
 //    units ahead.  Per k-step p the word's bits p of each byte give four 0/1 u8 A-fragment
 //    bytes; mma.m16n8k32 u8 x s8 gives S = sum bit * v over the unit exactly.
 //  * sum_k sign * v = 2 S - sum v; each unit adds 2^E (2 S - chunk sum) to the warp's fp32
-//    partial (times s1 in stage 2); tiles split between warps are finished in fixed order
-//    by the last one to arrive (tile_epilogue), so the result is deterministic.
+//    partial (times s1 in stage 2); tiles split between warps are added in shared memory
+//    after one CTA barrier, and tiles split between CTAs by the last CTA to arrive, both in
+//    a fixed order (cta_fix_finish), so the result is deterministic.
 //  * Both launches are programmatic dependents; only their first weight loads precede the
 //    wait for the previous kernel.
 #include <cstring>
+#include <type_traits>
 #include "lbq_common.cuh"
 #include "lbq_internal.h"
 #include "lbq_group_frag.cuh"
@@ -28,8 +30,7 @@
 
 namespace lbq {
 
-constexpr int kBinWarpsPerCta = 16;          // one CTA per SM: the stage input is prepared once per SM
-constexpr int kBinThreads = kBinWarpsPerCta * 32;
+constexpr int kBinPrepBatch = 4;             // prep chunks whose loads a warp issues together
 
 struct BinStageArgs {
     const uint8_t* signs;       // kernel sign layout, rows x cpad
@@ -43,7 +44,8 @@ struct BinStageArgs {
     unsigned* counters;
     int64_t rows, cols, cpad, ksb, n_tiles, total_units, total_warps;
     int M, maxc;
-    int sp, sv, se, szero;      // shared-memory offsets: planes, chunk sums, exponents, zero chunk
+    int sp, sv, se, szero;      // shared-memory offsets: planes, chunk sums, exponents, zero chunk,
+    int sfix;                   // CTA-level tile finish (CtaFix)
 };
 
 // Byte offset, in a 256-column chunk of a plane row, of column 32p + 16h + 4c + j: the
@@ -83,25 +85,30 @@ __device__ __forceinline__ PrepOut bin_quantize8(const float (&v)[8], int E) {
     return r;
 }
 
-// Lane's 8 stage-input values of token m, columns k0..k0+7 (zero past the last column).
+// Raw bits of the lane's 8 stage-input values of token m, columns k0..k0+7 (zero past the
+// last column): stage 1 x (r0) and s2 (r1), stage 2 the fp32 t (r0: 0..3, r1: 4..7).
 // The inputs may come from the previous kernel of the stream: read through L2.
-template <bool STAGE2, bool BF16>
-__device__ __forceinline__ void bin_load8(const BinStageArgs& a, int m, int64_t k0, float (&v)[8]) {
+template <bool STAGE2>
+__device__ __forceinline__ void bin_load_raw(const BinStageArgs& a, int m, int64_t k0, uint4& r0, uint4& r1) {
     if (k0 >= a.cols) {
-#pragma unroll
-        for (int e = 0; e < 8; e++) v[e] = 0.0f;
-        return;
-    }
-    if constexpr (STAGE2) {
-        const float4 p = __ldcg(reinterpret_cast<const float4*>(a.tin + (int64_t)m * a.cols + k0));
-        const float4 q = __ldcg(reinterpret_cast<const float4*>(a.tin + (int64_t)m * a.cols + k0 + 4));
-        v[0] = p.x; v[1] = p.y; v[2] = p.z; v[3] = p.w;
-        v[4] = q.x; v[5] = q.y; v[6] = q.z; v[7] = q.w;
+        r0 = r1 = make_uint4(0, 0, 0, 0);
+    } else if constexpr (STAGE2) {
+        r0 = __ldcg(reinterpret_cast<const uint4*>(a.tin + (int64_t)m * a.cols + k0));
+        r1 = __ldcg(reinterpret_cast<const uint4*>(a.tin + (int64_t)m * a.cols + k0 + 4));
     } else {
-        const uint4 xr = __ldcg(reinterpret_cast<const uint4*>(a.x + (int64_t)m * a.cols + k0));
-        const uint4 sr = __ldg(reinterpret_cast<const uint4*>(a.s2 + k0));
-        const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
-        const uint32_t sw[4] = {sr.x, sr.y, sr.z, sr.w};
+        r0 = __ldcg(reinterpret_cast<const uint4*>(a.x + (int64_t)m * a.cols + k0));
+        r1 = __ldg(reinterpret_cast<const uint4*>(a.s2 + k0));
+    }
+}
+
+template <bool STAGE2, bool BF16>
+__device__ __forceinline__ void bin_convert(const uint4& r0, const uint4& r1, float (&v)[8]) {
+    if constexpr (STAGE2) {
+        v[0] = __uint_as_float(r0.x); v[1] = __uint_as_float(r0.y); v[2] = __uint_as_float(r0.z); v[3] = __uint_as_float(r0.w);
+        v[4] = __uint_as_float(r1.x); v[5] = __uint_as_float(r1.y); v[6] = __uint_as_float(r1.z); v[7] = __uint_as_float(r1.w);
+    } else {
+        const uint32_t xw[4] = {r0.x, r0.y, r0.z, r0.w};
+        const uint32_t sw[4] = {r1.x, r1.y, r1.z, r1.w};
 #pragma unroll
         for (int e = 0; e < 8; e++) {
             const float xv = to_f32<BF16>((uint16_t)(xw[e / 2] >> (16 * (e & 1))));
@@ -111,8 +118,8 @@ __device__ __forceinline__ void bin_load8(const BinStageArgs& a, int m, int64_t 
     }
 }
 
-template <bool STAGE2, int D, bool BF16>
-__global__ void __launch_bounds__(kBinThreads, 1) k_binlr_ldg(const __grid_constant__ BinStageArgs a) {
+template <bool STAGE2, int D, int NW, bool BF16>
+__global__ void __launch_bounds__(NW * 32, 1) k_binlr_ldg(const __grid_constant__ BinStageArgs a) {
     constexpr int NB = 1;                      // M <= 4: hi/lo planes of 4 tokens in one n-block
     constexpr int PF = 16;                     // units prefetched into L2 before the wait
     extern __shared__ __align__(16) uint8_t smem[];
@@ -121,7 +128,7 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_binlr_ldg(const __grid_const
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
     const int64_t W = a.total_warps, S = a.total_units;
-    const int64_t wid = (int64_t)blockIdx.x * kBinWarpsPerCta + warp;
+    const int64_t wid = (int64_t)blockIdx.x * NW + warp;
     const int u_begin = (int)(wid < W ? wid * S / W : S);
     const int u_end = (int)(wid < W ? (wid + 1) * S / W : S);
     const bool has_work = u_begin < u_end;
@@ -142,37 +149,63 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_binlr_ldg(const __grid_const
     lptr += D * 512;
     if (lane < PF && u_begin + D + lane < u_end) l2_prefetch_bulk(lptr - 16 * lane + lane * 512, 512);
     if (threadIdx.x < 16) reinterpret_cast<uint4*>(smem + a.szero)[threadIdx.x] = make_uint4(0, 0, 0, 0);
+    // stage 2: the row scales of the warp's first tile (a weight, like the signs)
+    uint16_t s1h0 = 0, s1h1 = 0;
+    if constexpr (STAGE2) {
+        if (has_work) {
+            s1h0 = __ldg(a.s1 + (int64_t)ct * 16 + g);
+            s1h1 = __ldg(a.s1 + (int64_t)ct * 16 + g + 8);
+        }
+    }
     griddep_wait();
 
     // ---- prepare the stage input in one pass: per 256-column chunk one power-of-two scale,
     // the int8 planes and the exact chunk sum; the chunk order is rotated by the CTA index
     // so that the CTAs do not all read the same lines at once
     const int kch = (int)(a.cpad / kLdgChunk);
+    const int ntask = M * kch;                   // (token, chunk) pairs
     const int rot = (int)(blockIdx.x % (unsigned)kch);
     int* expo = reinterpret_cast<int*>(smem + a.se);
     int* vsum = reinterpret_cast<int*>(smem + a.sv);
-    for (int m = 0; m < M; m++) {
-        int8_t* row_h = reinterpret_cast<int8_t*>(smem + a.sp) + (int64_t)(2 * m) * a.cpad;
-        for (int cw = warp; cw < kch; cw += kBinWarpsPerCta) {
-            const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
-            float v[8];
-            bin_load8<STAGE2, BF16>(a, m, (int64_t)ch * kLdgChunk + 8 * lane, v);
-            const PrepOut r = bin_quantize8(v, ldg_fixed_point_exponent(warp_max_abs8(v)));
-            // elements 8 lane + 0..3 and + 4..7: columns 32p + 16h + 4c' + j
-            const int p = lane >> 2, h = (lane & 3) >> 1, c0 = 2 * (lane & 1);
-            int8_t* base = row_h + ch * kLdgChunk;
-            *reinterpret_cast<uint32_t*>(base + bin_plane_off(p, h, c0)) = r.hi.x;
-            *reinterpret_cast<uint32_t*>(base + bin_plane_off(p, h, c0 + 1)) = r.hi.y;
-            *reinterpret_cast<uint32_t*>(base + a.cpad + bin_plane_off(p, h, c0)) = r.lo.x;
-            *reinterpret_cast<uint32_t*>(base + a.cpad + bin_plane_off(p, h, c0 + 1)) = r.lo.y;
-            if (lane == 0) {
-                vsum[m * kch + ch] = r.gsum;
-                expo[m * kch + ch] = r.E;
+    // a warp's chunks are independent: issue the loads of kBinPrepBatch of them together
+    for (int t0 = warp; t0 < ntask; t0 += NW * kBinPrepBatch) {
+        uint4 r0[kBinPrepBatch], r1[kBinPrepBatch];
+#pragma unroll
+        for (int j = 0; j < kBinPrepBatch; j++) {
+            const int t = t0 + j * NW;
+            if (t < ntask) {
+                const int m = t / kch, cw = t - m * kch;
+                const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
+                bin_load_raw<STAGE2>(a, m, (int64_t)ch * kLdgChunk + 8 * lane, r0[j], r1[j]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kBinPrepBatch; j++) {
+            const int t = t0 + j * NW;
+            if (t < ntask) {
+                const int m = t / kch, cw = t - m * kch;
+                const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
+                float v[8];
+                bin_convert<STAGE2, BF16>(r0[j], r1[j], v);
+                const PrepOut r = bin_quantize8(v, ldg_fixed_point_exponent(warp_max_abs8(v)));
+                // elements 8 lane + 0..3 and + 4..7: columns 32p + 16h + 4c' + j
+                const int p = lane >> 2, h = (lane & 3) >> 1, c0 = 2 * (lane & 1);
+                int8_t* base = reinterpret_cast<int8_t*>(smem + a.sp) + (int64_t)(2 * m) * a.cpad + ch * kLdgChunk;
+                *reinterpret_cast<uint32_t*>(base + bin_plane_off(p, h, c0)) = r.hi.x;
+                *reinterpret_cast<uint32_t*>(base + bin_plane_off(p, h, c0 + 1)) = r.hi.y;
+                *reinterpret_cast<uint32_t*>(base + a.cpad + bin_plane_off(p, h, c0)) = r.lo.x;
+                *reinterpret_cast<uint32_t*>(base + a.cpad + bin_plane_off(p, h, c0 + 1)) = r.lo.y;
+                if (lane == 0) {
+                    vsum[m * kch + ch] = r.gsum;
+                    expo[m * kch + ch] = r.E;
+                }
             }
         }
     }
     __syncthreads();
-    if (!has_work) return;
+    const CtaFix fix = cta_fix_at(smem + a.sfix, NW, M);
+    cta_fix_clear(fix, warp, lane);
+    const int head_tile = ct;
 
     // B-fragment row of this lane (plane g: token g / 2, hi or lo) and its token's sums
     const bool pv = g < 2 * M;
@@ -198,41 +231,49 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_binlr_ldg(const __grid_const
                     lptr += 512;
                 }
                 const int8_t* pr = prow + csb * pstep;
-                // S = sum over the unit of bit * v, exactly: 0/1 A bytes of k-step p
-                int s[4];
+                // S = sum over the unit of bit * v, exactly: 0/1 A bytes of k-step p; the even
+                // and the odd k-steps accumulate in two independent chains
+                int se[4], so[4];
 #pragma unroll
                 for (int p = 0; p < 8; p += 2) {
                     const uint4 bq = *reinterpret_cast<const uint4*>(pr + 64 * (p >> 1));
-#pragma unroll
-                    for (int q = 0; q < 2; q++) {
-                        const int sh = p + q;
-                        const uint32_t a0 = (w.x >> sh) & 0x01010101u, a1 = (w.y >> sh) & 0x01010101u;
-                        const uint32_t a2 = (w.z >> sh) & 0x01010101u, a3 = (w.w >> sh) & 0x01010101u;
-                        if (sh == 0) mma_16832_u8s8_zc(s, a0, a1, a2, a3, bq.x, bq.y);
-                        else mma_16832_u8s8(s, a0, a1, a2, a3, q ? bq.z : bq.x, q ? bq.w : bq.y);
+                    const uint32_t a0 = (w.x >> p) & 0x01010101u, a1 = (w.y >> p) & 0x01010101u;
+                    const uint32_t a2 = (w.z >> p) & 0x01010101u, a3 = (w.w >> p) & 0x01010101u;
+                    const uint32_t b0 = (w.x >> (p + 1)) & 0x01010101u, b1 = (w.y >> (p + 1)) & 0x01010101u;
+                    const uint32_t b2 = (w.z >> (p + 1)) & 0x01010101u, b3 = (w.w >> (p + 1)) & 0x01010101u;
+                    if (p == 0) {
+                        mma_16832_u8s8_zc(se, a0, a1, a2, a3, bq.x, bq.y);
+                        mma_16832_u8s8_zc(so, b0, b1, b2, b3, bq.z, bq.w);
+                    } else {
+                        mma_16832_u8s8(se, a0, a1, a2, a3, bq.x, bq.y);
+                        mma_16832_u8s8(so, b0, b1, b2, b3, bq.z, bq.w);
                     }
                 }
                 // sum_k sign * v = 2 S - sum v, times this chunk's 2^E; columns 2c (hi), 2c + 1 (lo)
                 const int vs = vrow[csb * vstep];
                 const float sc = ldg_exp2i(erow[csb * vstep]);
-                part0 = fmaf(sc, (float)(2 * (256 * s[0] + s[1]) - vs), part0);
-                part1 = fmaf(sc, (float)(2 * (256 * s[2] + s[3]) - vs), part1);
+                part0 = fmaf(sc, (float)(2 * (256 * (se[0] + so[0]) + se[1] + so[1]) - vs), part0);
+                part1 = fmaf(sc, (float)(2 * (256 * (se[2] + so[2]) + se[3] + so[3]) - vs), part1);
                 if (csb == ksb - 1 || u == u_end - 1) {
-                    float part[NB][2];
+                    float part[NB][2];   // [0][0]: row g, [0][1]: row g + 8 of token c
                     part[0][0] = tv ? part0 : 0.0f;
                     part[0][1] = tv ? part1 : 0.0f;
-                    const int64_t row = (int64_t)ct * 16 + g;
                     if constexpr (STAGE2) {
-                        part[0][0] *= __half2float(__ushort_as_half(a.s1[row]));
-                        part[0][1] *= __half2float(__ushort_as_half(a.s1[row + 8]));
+                        part[0][0] *= __half2float(__ushort_as_half(s1h0));
+                        part[0][1] *= __half2float(__ushort_as_half(s1h1));
+                        // the next tile's row scales, a tile ahead of their use
+                        if (ct + 1 < a.n_tiles) {
+                            s1h0 = __ldg(a.s1 + (int64_t)(ct + 1) * 16 + g);
+                            s1h1 = __ldg(a.s1 + (int64_t)(ct + 1) * 16 + g + 8);
+                        }
                     }
                     const bool full = tile_first_u >= u_begin && csb == ksb - 1;
-                    if constexpr (STAGE2)
-                        tile_epilogue<NB>(part, full, M, a.rows, ct, ct, (int64_t)ct * ksb, ksb, S, W, wid, a.partials,
-                                          a.counters, a.maxc, a.y);
-                    else
-                        tile_epilogue_f32<NB>(part, full, M, a.rows, ct, ct, (int64_t)ct * ksb, ksb, S, W, wid,
-                                              a.partials, a.counters, a.maxc, a.tout);
+                    if (full) {
+                        if constexpr (STAGE2) tile_store_full<NB>(part, M, a.rows, ct, a.y);
+                        else tile_store_full<NB>(part, M, a.rows, ct, a.tout);
+                    } else {
+                        cta_fix_put<NB>(fix, warp, ct == head_tile ? 0 : 1, ct, part, M);
+                    }
                     part0 = part1 = 0.0f;
                     tile_first_u = u + 1;
                 }
@@ -243,6 +284,23 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_binlr_ldg(const __grid_const
             }
         }
     }
+
+    // ---- partial tiles: CTA sums in shared memory, CTA-crossing tiles by ticket
+    __syncthreads();
+    const int64_t cw0 = (int64_t)blockIdx.x * NW, cw1 = min(cw0 + NW, W);
+    const int64_t C0 = cw0 < W ? cw0 * S / W : S, C1 = cw0 < W ? cw1 * S / W : S;
+    using Y = typename std::conditional<STAGE2, uint16_t, float>::type;
+    Y* yout;
+    if constexpr (STAGE2) yout = a.y;
+    else yout = a.tout;
+    cta_fix_finish<Y>(fix, NW, warp, M, u_begin, C0, C1, S, W, blockIdx.x, a.partials, a.counters, a.maxc,
+                      [&](int T, int64_t& first_u, int64_t& units, Y*& y, int64_t& n, int64_t& row0) {
+                          first_u = (int64_t)T * ksb;
+                          units = ksb;
+                          y = yout;
+                          n = a.rows;
+                          row0 = (int64_t)T * 16;
+                      });
 }
 
 // ------------------------------------------------------------------ host side
@@ -252,12 +310,16 @@ struct BinLdgPlan {
     size_t part1, part2, t_off, bytes;
 };
 
+// Warps per CTA and register ring depth of the sign stream (one CTA per SM: the stage
+// input is prepared once per SM).
+constexpr int kBinNW = 16, kBinD = 8;
+
 static void bin_stage_plan(int64_t rows, int64_t cpad, int64_t& units, int64_t& warps, int& grid, int& maxc) {
     const int64_t ksb = cpad / kLdgChunk;
     units = rows / 16 * ksb;
     constexpr int64_t kMinUnitsPerWarp = 4;
-    grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sm_count(), ceil_div(units, kBinWarpsPerCta * kMinUnitsPerWarp)));
-    warps = std::min<int64_t>((int64_t)grid * kBinWarpsPerCta, std::max<int64_t>(units, 1));
+    grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sm_count(), ceil_div(units, kBinNW * kMinUnitsPerWarp)));
+    warps = std::min<int64_t>((int64_t)grid * kBinNW, std::max<int64_t>(units, 1));
     maxc = (int)(ceil_div(ksb * warps, std::max<int64_t>(units, 1)) + 2);
 }
 
@@ -272,9 +334,11 @@ static BinLdgPlan bin_ldg_plan(int64_t M, int64_t d_out, int64_t d_in, int64_t r
     return pl;
 }
 
+static int bin_fix_bytes(int64_t M) { return al16(kBinNW * 2 * 16 * M * 4 + kBinNW * 2 * 4); }
+
 static int bin_smem_bytes(int64_t M, int64_t cpad) {
-    // planes [2M][cpad] | chunk sums [M][cpad/256] | chunk exponents [M][cpad/256] | zero chunk
-    return al16(2 * M * cpad) + 2 * al16(M * (cpad / kLdgChunk) * 4) + 256;
+    // planes [2M][cpad] | chunk sums [M][cpad/256] | chunk exponents [M][cpad/256] | zero chunk | CTA finish
+    return al16(2 * M * cpad) + 2 * al16(M * (cpad / kLdgChunk) * 4) + 256 + bin_fix_bytes(M);
 }
 
 bool gemv_binlr_ldg_supported(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
@@ -291,11 +355,10 @@ size_t gemv_binlr_ldg_ws_bytes(int64_t M, int64_t d_out, int64_t d_in, int64_t r
 
 template <bool STAGE2, bool BF16>
 static lbq_status launch_bin_stage(const BinStageArgs& a, int grid, int smem, cudaStream_t st) {
-    constexpr int D = 8;
-    constexpr auto kern = k_binlr_ldg<STAGE2, D, BF16>;
+    constexpr auto kern = k_binlr_ldg<STAGE2, kBinD, kBinNW, BF16>;
     const lbq_status s = ldg_smem_attr<kern>(200 * 1024);
     if (s != LBQ_OK) return s;
-    return launch_pdl(kern, grid, kBinThreads, (size_t)smem, st, a);
+    return launch_pdl(kern, grid, kBinNW * 32, (size_t)smem, st, a);
 }
 
 lbq_status launch_gemv_binlr_ldg(const void* x, bool bf16, int64_t M, const void* U, const void* Vt, const void* s1,
@@ -332,6 +395,7 @@ lbq_status launch_gemv_binlr_ldg(const void* x, bool bf16, int64_t M, const void
         a.sv = al16(2 * M * a.cpad);
         a.se = a.sv + al16(M * a.ksb * 4);
         a.szero = a.se + al16(M * a.ksb * 4);
+        a.sfix = a.szero + 256;
         const int smem = bin_smem_bytes(M, a.cpad);
         const int grid = st2 ? pl.grid2 : pl.grid1;
         lbq_status s;

@@ -209,6 +209,14 @@ __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
 __device__ __forceinline__ void named_barrier(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Ticket increment with acquire-release semantics at GPU scope: the caller's earlier writes
+// (and those ordered before it by a warp or CTA barrier) are visible to whoever reads the
+// incremented value, and the writes of earlier incrementers are visible to the caller.
+__device__ __forceinline__ unsigned atomic_add_acq_rel_gpu(unsigned* p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
 // Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) from global memory into L2.
 __device__ __forceinline__ void l2_prefetch_bulk(const void* src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");

@@ -108,6 +108,126 @@ __device__ __forceinline__ void tile_epilogue_any(const float (&acc)[NB][2], boo
     }
 }
 
+// ------------------------------------------------------------------ CTA-level tile finish
+// Warp-level stream-K over a CTA's contiguous unit range leaves each warp at most two
+// partial tiles: the tile of its first unit (slot 0) and, if different, the tile of its
+// last unit (slot 1).  The warps park those partial sums in shared memory; after one CTA
+// barrier the CTA's first contributing warp of each tile adds them in warp order.  A tile
+// that lies inside the CTA's range is stored at once; one shared with other CTAs goes
+// through the global ticket (the last of its CTAs adds the CTA sums in CTA order), so at
+// most two tiles per CTA pay for a GPU-scope atomic, and the sum order is fixed.
+struct CtaFix {
+    float* val;     // [NW][2][16 * M] partial sums, element tok * 16 + row
+    int* tile;      // [NW][2] tile index of each slot, -1 if unused
+};
+
+__device__ __forceinline__ size_t cta_fix_bytes(int nw, int M) {
+    return (size_t)nw * 2 * 16 * M * 4 + (size_t)nw * 2 * 4;
+}
+__device__ __forceinline__ CtaFix cta_fix_at(uint8_t* base, int nw, int M) {
+    CtaFix f;
+    f.val = reinterpret_cast<float*>(base);
+    f.tile = reinterpret_cast<int*>(base + (size_t)nw * 2 * 16 * M * 4);
+    return f;
+}
+__device__ __forceinline__ void cta_fix_clear(const CtaFix& f, int warp, int lane) {
+    if (lane < 2) f.tile[warp * 2 + lane] = -1;
+}
+// Park a warp's partial tile (fragment layout of tile_epilogue) in slot k.
+template <int NB>
+__device__ __forceinline__ void cta_fix_put(const CtaFix& f, int warp, int k, int64_t tile, const float (&acc)[NB][2],
+                                            int M) {
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    float* v = f.val + (warp * 2 + k) * 16 * M;
+#pragma unroll
+    for (int nb = 0; nb < NB; nb++) {
+        const int tok = 4 * nb + c;
+        if (tok < M) {
+            v[tok * 16 + g] = acc[nb][0];
+            v[tok * 16 + g + 8] = acc[nb][1];
+        }
+    }
+    if (lane == 0) f.tile[warp * 2 + k] = (int)tile;
+}
+// Store a full tile straight from the fragments.
+template <int NB, class Y>
+__device__ __forceinline__ void tile_store_full(const float (&acc)[NB][2], int M, int64_t n, int64_t tile, Y* y) {
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int nb = 0; nb < NB; nb++) {
+        const int tok = 4 * nb + c;
+        if (tok < M) {
+            store_out(y + (int64_t)tok * n + tile * 16 + g, acc[nb][0]);
+            store_out(y + (int64_t)tok * n + tile * 16 + g + 8, acc[nb][1]);
+        }
+    }
+}
+// After the CTA barrier: finish the tiles this warp owns.  info(T, first_u, units, y, n, row0)
+// describes tile T: its units [first_u, first_u + units) in the launch's unit list, and the
+// output rows y[tok * n + row0 + 0..15].  The launch's W warps split S units evenly
+// (warp w: [w S / W, (w + 1) S / W)), NW per CTA; u_begin is this warp's first unit,
+// [C0, C1) the CTA's range and cta its index.
+template <class Y, class Info>
+__device__ __forceinline__ void cta_fix_finish(const CtaFix& f, int NW, int warp, int M, int64_t u_begin, int64_t C0,
+                                               int64_t C1, int64_t S, int64_t W, int64_t cta,
+                                               float* __restrict__ partials, unsigned* __restrict__ counters, int maxc,
+                                               Info info) {
+    const int lane = threadIdx.x & 31;
+    const int E = 16 * M;
+#pragma unroll 1
+    for (int k = 0; k < 2; k++) {
+        const int T = f.tile[warp * 2 + k];
+        if (T < 0) continue;
+        int64_t first_u, units, n, row0;
+        Y* y;
+        info(T, first_u, units, y, n, row0);
+        if (k == 0 && warp > 0 && first_u < u_begin) continue;   // an earlier warp of this CTA owns it
+        int w_end = warp + 1;
+        while (w_end < NW && f.tile[w_end * 2] == T) w_end++;
+        const bool inside = first_u >= C0 && first_u + units <= C1;
+        int64_t cf = 0, count = 1;
+        float* p0 = nullptr;
+        if (!inside) {
+            cf = (((first_u + 1) * W - 1) / S) / NW;
+            const int64_t cl = (((first_u + units) * W - 1) / S) / NW;
+            count = cl - cf + 1;
+            p0 = partials + (int64_t)T * maxc * E;
+        }
+        for (int e = lane; e < E; e += 32) {
+            float s = f.val[(warp * 2 + k) * E + e];
+            for (int w2 = warp + 1; w2 < w_end; w2++) s += f.val[(w2 * 2) * E + e];
+            if (inside) store_out(y + (int64_t)(e / 16) * n + row0 + (e % 16), s);
+            else __stcg(p0 + (cta - cf) * E + e, s);
+        }
+        if (inside) continue;
+        __syncwarp();
+        unsigned old = 0;
+        if (lane == 0) old = atomic_add_acq_rel_gpu(counters + T, 1u);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old == (unsigned)(count - 1)) {
+            __syncwarp();   // orders every lane's slot loads after lane 0's acquire
+            // the slots' loads are independent: batches of 8, added in CTA order
+            for (int e = lane; e < E; e += 32) {
+                float s = 0.0f;
+                int sl = 0;
+                for (; sl + 8 <= count; sl += 8) {
+                    float v[8];
+#pragma unroll
+                    for (int j = 0; j < 8; j++) v[j] = __ldcg(p0 + (sl + j) * (int64_t)E + e);
+#pragma unroll
+                    for (int j = 0; j < 8; j++) s += v[j];
+                }
+                for (; sl < count; sl++) s += __ldcg(p0 + sl * (int64_t)E + e);
+                store_out(y + (int64_t)(e / 16) * n + row0 + (e % 16), s);
+            }
+            __syncwarp();
+            if (lane == 0) counters[T] = 0u;
+        }
+    }
+}
+
 template <int NB>
 __device__ __forceinline__ void tile_epilogue(const float (&acc)[NB][2], bool full, int M, int64_t n, int64_t tile,
                                               int64_t gtile, int64_t first_u, int64_t units_per_rb, int64_t S_total,
