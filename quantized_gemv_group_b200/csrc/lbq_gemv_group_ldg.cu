@@ -9,25 +9,27 @@
 //  * Work list: the (16-row tile, 256-wide k superblock) units of up to kMaxGemvProblems
 //    products of one bit width and group size (e.g. the q/k/v or gate/up projections of
 //    a decoder block), tile-major.  Every warp of the grid takes an equal contiguous
-//    slice of it ("stream-K" at warp granularity), so all warps finish together; a tile
-//    split between warps is finished by the last one to arrive (tile_epilogue, fixed
-//    order, deterministic).
+//    slice of it ("stream-K" at warp granularity), so all warps finish together.  A tile
+//    split between warps of one CTA is added in shared memory after one CTA barrier; a
+//    tile split between CTAs by the last CTA to arrive at its ticket (cta_fix_finish):
+//    fixed order, deterministic, at most two GPU-scope tickets per CTA.
 //  * Each warp streams its units' packed words straight into registers with 128-bit
 //    non-coherent loads (evict-first in L2), keeping D units in flight: one unit is the
 //    lane's 16 * B bytes of a tile's 512 * B-byte superblock block, already in mma
 //    fragment order.  Warps never wait for one another, so a warp stalled on compute or
 //    on a scale load leaves the other warps' loads in flight.
-//  * A prep kernel turns every distinct activation row into 16-bit fixed point with one
-//    power-of-two scale 2^E per token and 256-wide chunk (|v| <= 32639), stored as two
-//    int8 planes hi, lo (v = 256 hi + lo) in B-fragment order, plus exact per-group sums
-//    of v.  The warps read these through L1.
+//  * Every distinct activation row becomes 16-bit fixed point with one power-of-two
+//    scale 2^E per token and 256-wide chunk (|v| <= 32639), stored as two int8 planes
+//    hi, lo (v = 256 hi + lo) in B-fragment order, plus exact per-group sums of v.  For
+//    one token block each CTA prepares them in its own shared memory right after the
+//    wait; otherwise a prep kernel writes them to the workspace, read through L2.
 //  * Per k-step the lane masks its words into u8 A fragments (one LOP per four codes)
 //    and runs mma.m16n8k32 u8 x s8 -> s32 with the hi and lo planes side by side in N.
 //    Per group the exact integer sum S = sum q v becomes sum (q - z) v = S - z sum(v),
 //    scaled by s into an fp32 chunk accumulator, which is scaled by 2^E once per chunk.
-//  * Both kernels are launched as programmatic dependents: the GEMV's first weight
-//    loads are issued before it waits for the prep kernel (griddepcontrol.wait), and the
-//    prep kernel waits for the previous kernel in the stream before reading x.  Packed
+//  * The kernels are launched as programmatic dependents: the GEMV's first weight
+//    loads are issued before it waits for the previous kernel (griddepcontrol.wait), and
+//    x is read only after that wait.  Packed
 //    weights, scales and zeros must therefore not be written by a kernel that signals
 //    programmatic completion early.
 // Group codes: "TurboQuant: cuantizar modelos grandes para que quepan en local",
@@ -59,6 +61,7 @@ struct LdgArgs {
     int count, M, maxc;
     int sring;              // byte offset of the scale/zero rings in shared memory
     int szero;              // byte offset of a 256-byte zero chunk in shared memory
+    int sfix;               // byte offset of the CTA-level tile finish (CtaFix)
 };
 
 constexpr int kScaleRing = 6;               // units of scales/zeros in flight per warp
@@ -317,7 +320,9 @@ __global__ void __launch_bounds__(NW * 32, 1)
         }
     }
     __syncthreads();
-    if (!has_work) return;
+    const CtaFix fix = cta_fix_at(smem + a.sfix, NW, M);
+    cta_fix_clear(fix, warp, lane);
+    const int head_gtile = (int)a.p[cp].tile_begin + ct;
 
     // per-problem byte offsets, from one base, of this lane's plane rows, group sums and
     // exponents; padded rows and tokens point at the zero chunk with a zero stride
@@ -443,8 +448,9 @@ __global__ void __launch_bounds__(NW * 32, 1)
                 const LdgProblem& P = a.p[cp];
                 if (csb == P.ksb - 1 || u == u_end - 1) {
                     const bool full = tile_first_u >= u_begin && csb == P.ksb - 1;
-                    tile_epilogue<NB>(acc, full, M, P.n, ct, P.tile_begin + ct, P.unit_begin + ct * P.ksb, P.ksb, S, W,
-                                      wid, a.partials, a.counters, a.maxc, P.y);
+                    const int gt = (int)P.tile_begin + ct;
+                    if (full) tile_store_full<NB>(acc, M, P.n, ct, P.y);
+                    else cta_fix_put<NB>(fix, warp, gt == head_gtile ? 0 : 1, gt, acc, M);
 #pragma unroll
                     for (int nb = 0; nb < NB; nb++) acc[nb][0] = acc[nb][1] = 0.0f;
                     tile_first_u = u + 1;
@@ -460,6 +466,23 @@ __global__ void __launch_bounds__(NW * 32, 1)
             }
         }
     }
+
+    // ---- partial tiles: CTA sums in shared memory, CTA-crossing tiles by ticket
+    __syncthreads();
+    const int64_t cw0 = (int64_t)blockIdx.x * NW, cw1 = min(cw0 + NW, W);
+    const int64_t C0 = cw0 < W ? cw0 * S / W : S, C1 = cw0 < W ? cw1 * S / W : S;
+    cta_fix_finish<uint16_t>(fix, NW, warp, M, u_begin, C0, C1, S, W, blockIdx.x, a.partials, a.counters, a.maxc,
+                             [&](int T, int64_t& first_u, int64_t& units, uint16_t*& y, int64_t& n, int64_t& row0) {
+                                 int q = 0;
+                                 while (q + 1 < a.count && T >= a.p[q + 1].tile_begin) q++;
+                                 const LdgProblem& Q = a.p[q];
+                                 const int64_t t = T - Q.tile_begin;
+                                 first_u = Q.unit_begin + t * Q.ksb;
+                                 units = Q.ksb;
+                                 y = Q.y;
+                                 n = Q.n;
+                                 row0 = t * 16;
+                             });
 }
 
 // ------------------------------------------------------------------ host side
@@ -646,10 +669,12 @@ lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count,
     // prepared activations in each CTA's shared memory when they fit, else one prep launch;
     // the scale/zero rings follow them (or start the shared memory)
     const int ring = shape.NW * kScaleRing * scale_slot_bytes(group);
-    const bool smemp = NB == 1 && soff + ring + 256 <= kLdgSmemBudget;
+    const int fixb = al16(shape.NW * 2 * 16 * M * 4 + shape.NW * 2 * 4);
+    const bool smemp = NB == 1 && soff + ring + 256 + fixb <= kLdgSmemBudget;
     args.sring = smemp ? al16(soff) : 0;
     args.szero = args.sring + ring;
-    const int smem = args.szero + 256;
+    args.sfix = args.szero + 256;
+    const int smem = args.sfix + fixb;
     if (!smemp) {
         const int pgrid = (int)ceil_div(pw, (int64_t)8);
         lbq_status s;
