@@ -334,7 +334,7 @@ static BinLdgPlan bin_ldg_plan(int64_t M, int64_t d_out, int64_t d_in, int64_t r
     return pl;
 }
 
-static int bin_fix_bytes(int64_t M) { return al16(kBinNW * 2 * 16 * M * 4 + kBinNW * 2 * 4); }
+static int bin_fix_bytes(int64_t M) { return al16((int64_t)cta_fix_bytes(kBinNW, (int)M)); }
 
 static int bin_smem_bytes(int64_t M, int64_t cpad) {
     // planes [2M][cpad] | chunk sums [M][cpad/256] | chunk exponents [M][cpad/256] | zero chunk | CTA finish

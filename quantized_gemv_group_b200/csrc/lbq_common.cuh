@@ -209,6 +209,25 @@ __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
 __device__ __forceinline__ void named_barrier(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Thread-block clusters: this CTA's rank, the cluster-window address of shared-memory
+// address `saddr` in the CTA of rank `rank`, a store there, and a barrier of every thread
+// of the cluster (release / acquire: shared-memory stores before it are visible after it).
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_map_smem(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 // Ticket increment with acquire-release semantics at GPU scope: the caller's earlier writes
 // (and those ordered before it by a warp or CTA barrier) are visible to whoever reads the
 // incremented value, and the writes of earlier incrementers are visible to the caller.

@@ -57,14 +57,24 @@ struct LdgArgs {
     LdgProblem p[kMaxGemvProblems];
     float* partials;
     unsigned* counters;
-    int64_t total_units, total_warps;
+    int64_t total_units, total_warps, total_tiles;
     int count, M, maxc;
+    int pair;               // 1: clusters of two CTAs, each pair a whole number of tiles
     int sring;              // byte offset of the scale/zero rings in shared memory
     int szero;              // byte offset of a 256-byte zero chunk in shared memory
     int sfix;               // byte offset of the CTA-level tile finish (CtaFix)
 };
 
+// First unit of launch-wide tile T (total_units for T = total_tiles).
+__device__ __forceinline__ int64_t ldg_tile_first_unit(const LdgArgs& a, int64_t T) {
+    if (T >= a.total_tiles) return a.total_units;
+    int q = 0;
+    while (q + 1 < a.count && T >= a.p[q + 1].tile_begin) q++;
+    return a.p[q].unit_begin + (T - a.p[q].tile_begin) * a.p[q].ksb;
+}
+
 constexpr int kScaleRing = 6;               // units of scales/zeros in flight per warp
+constexpr int kPrepBatch = 4;               // activation chunks whose loads a warp issues together
 
 // Bytes of one unit's scale/zero slot: 2 arrays x 16 rows x (256 / GROUP) fp16.
 constexpr int scale_slot_bytes(int group) { return 64 * (kLdgChunk / group); }
@@ -216,11 +226,35 @@ __global__ void __launch_bounds__(NW * 32, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
     const int64_t W = a.total_warps, S = a.total_units;
-    const int64_t wid = (int64_t)blockIdx.x * NW + warp;
-    // warps past the W that share the list (grid * 8 may exceed it) take no units;
-    // unit indices fit 32 bits (the host caps the list)
-    const int u_begin = (int)(wid < W ? wid * S / W : S);
-    const int u_end = (int)(wid < W ? (wid + 1) * S / W : S);
+    // this warp's units [u_begin, u_end) and the CTA's [C0, C1); unit indices fit 32 bits
+    // (the host caps the list)
+    int64_t ub, ue, C0, C1;
+    if (a.pair) {
+        // pair p of P takes tiles [p NT / P, (p + 1) NT / P); min(2 NW, its units) warps of
+        // the pair split them evenly, the other warps take none
+        const int64_t P = gridDim.x >> 1, p = blockIdx.x >> 1, rank = blockIdx.x & 1;
+        const int64_t U0 = ldg_tile_first_unit(a, p * a.total_tiles / P);
+        const int64_t U1 = ldg_tile_first_unit(a, (p + 1) * a.total_tiles / P);
+        const int64_t n = U1 - U0, Wp = n < 2 * NW ? n : (int64_t)(2 * NW), wp = rank * NW + warp;
+        if (n == 0) {
+            ub = ue = C0 = C1 = U0;
+        } else {
+            ub = wp < Wp ? U0 + wp * n / Wp : U1;
+            ue = wp < Wp ? U0 + (wp + 1) * n / Wp : U1;
+            C0 = U0 + (rank * NW < Wp ? rank * NW : Wp) * n / Wp;
+            C1 = U0 + ((rank + 1) * NW < Wp ? (rank + 1) * NW : Wp) * n / Wp;
+        }
+    } else {
+        // warps past the W that share the list take no units
+        const int64_t wid = (int64_t)blockIdx.x * NW + warp;
+        ub = wid < W ? wid * S / W : S;
+        ue = wid < W ? (wid + 1) * S / W : S;
+        const int64_t cw0 = (int64_t)blockIdx.x * NW, cw1 = min(cw0 + NW, W);
+        C0 = cw0 < W ? cw0 * S / W : S;
+        C1 = cw0 < W ? cw1 * S / W : S;
+    }
+    const int u_begin = (int)ub;
+    const int u_end = (int)ue;
     const int M = a.M;
     const uint64_t pol = l2_policy_evict_first();
 
@@ -277,12 +311,10 @@ __global__ void __launch_bounds__(NW * 32, 1)
         if (u_begin + i < u_end) issue_scales(i);
         cp_async_commit();
     }
-    // prologue: the first D units' weights (into registers) and the next PF (into L2)
-    // do not depend on the previous kernels
-#pragma unroll
-    for (int d = 0; d < D; d++)
-        if (u_begin + d < u_end) load_next(wb[d]);
-    if (lane < PF && u_begin + D + lane < u_end && lleft > lane)
+    // prologue: the first D + PF units into L2.  Bulk prefetches hold no registers and block
+    // no issue slot, so the wait and the activation prep start at once while HBM streams;
+    // the register ring is filled (from L2) after the prep
+    if (lane < D + PF && u_begin + lane < u_end && lleft > lane)
         l2_prefetch_bulk(lptr - 16 * lane + (int64_t)lane * (512 * B), 512 * B);
     // zeroed chunk that padded plane rows and tokens read instead of branching
     const int8_t* zero;
@@ -307,19 +339,37 @@ __global__ void __launch_bounds__(NW * 32, 1)
                 int8_t* row_h = reinterpret_cast<int8_t*>(smem + Q.sp) + (int64_t)(2 * m) * k32;
                 float* xs = reinterpret_cast<float*>(smem + Q.sx) + m * (k32 / GROUP);
                 int* ex = reinterpret_cast<int*>(smem + Q.se) + m * kch;
-                for (int cw = warp; cw < kch; cw += NW) {
-                    const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
-                    const PrepOut r = prep_chunk<GROUP, BF16>(xm + ch * kLdgChunk, lane);
-                    *reinterpret_cast<uint2*>(row_h + ch * kLdgChunk + plane_off(lane)) = r.hi;
-                    *reinterpret_cast<uint2*>(row_h + k32 + ch * kLdgChunk + plane_off(lane)) = r.lo;
-                    constexpr int LPG = GROUP / 8;
-                    if (lane % LPG == 0) xs[ch * (kLdgChunk / GROUP) + lane / LPG] = (float)r.gsum;
-                    if (lane == 0) ex[ch] = r.E;
+                // a warp's chunks are independent: issue kPrepBatch loads of x together
+                constexpr int PB = kPrepBatch;
+                for (int cw0 = warp; cw0 < kch; cw0 += NW * PB) {
+                    uint4 raw[PB];
+#pragma unroll
+                    for (int j = 0; j < PB; j++) {
+                        const int cw = cw0 + j * NW;
+                        const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
+                        if (cw < kch) raw[j] = prep_load(xm + ch * kLdgChunk, lane);
+                    }
+#pragma unroll
+                    for (int j = 0; j < PB; j++) {
+                        const int cw = cw0 + j * NW;
+                        if (cw < kch) {
+                            const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
+                            const PrepOut r = prep_convert<GROUP, BF16>(raw[j]);
+                            *reinterpret_cast<uint2*>(row_h + ch * kLdgChunk + plane_off(lane)) = r.hi;
+                            *reinterpret_cast<uint2*>(row_h + k32 + ch * kLdgChunk + plane_off(lane)) = r.lo;
+                            constexpr int LPG = GROUP / 8;
+                            if (lane % LPG == 0) xs[ch * (kLdgChunk / GROUP) + lane / LPG] = (float)r.gsum;
+                            if (lane == 0) ex[ch] = r.E;
+                        }
+                    }
                 }
             }
         }
     }
     __syncthreads();
+#pragma unroll
+    for (int d = 0; d < D; d++)
+        if (u_begin + d < u_end) load_next(wb[d]);
     const CtaFix fix = cta_fix_at(smem + a.sfix, NW, M);
     cta_fix_clear(fix, warp, lane);
     const int head_gtile = (int)a.p[cp].tile_begin + ct;
@@ -467,22 +517,28 @@ __global__ void __launch_bounds__(NW * 32, 1)
         }
     }
 
-    // ---- partial tiles: CTA sums in shared memory, CTA-crossing tiles by ticket
+    // ---- partial tiles: CTA sums in shared memory; a tile shared with another CTA goes
+    // by ticket, or in pair mode across the cluster barrier to rank 0
     __syncthreads();
-    const int64_t cw0 = (int64_t)blockIdx.x * NW, cw1 = min(cw0 + NW, W);
-    const int64_t C0 = cw0 < W ? cw0 * S / W : S, C1 = cw0 < W ? cw1 * S / W : S;
+    auto info = [&](int T, int64_t& first_u, int64_t& units, uint16_t*& y, int64_t& n, int64_t& row0) {
+        int q = 0;
+        while (q + 1 < a.count && T >= a.p[q + 1].tile_begin) q++;
+        const LdgProblem& Q = a.p[q];
+        const int64_t t = T - Q.tile_begin;
+        first_u = Q.unit_begin + t * Q.ksb;
+        units = Q.ksb;
+        y = Q.y;
+        n = Q.n;
+        row0 = t * 16;
+    };
+    PairKeep keep;
     cta_fix_finish<uint16_t>(fix, NW, warp, M, u_begin, C0, C1, S, W, blockIdx.x, a.partials, a.counters, a.maxc,
-                             [&](int T, int64_t& first_u, int64_t& units, uint16_t*& y, int64_t& n, int64_t& row0) {
-                                 int q = 0;
-                                 while (q + 1 < a.count && T >= a.p[q + 1].tile_begin) q++;
-                                 const LdgProblem& Q = a.p[q];
-                                 const int64_t t = T - Q.tile_begin;
-                                 first_u = Q.unit_begin + t * Q.ksb;
-                                 units = Q.ksb;
-                                 y = Q.y;
-                                 n = Q.n;
-                                 row0 = t * 16;
-                             });
+                             info, a.pair ? 1 + (int)(blockIdx.x & 1) : 0, &keep);
+    if (a.pair) {
+        __syncwarp();
+        cluster_sync_all();          // every thread of both CTAs: no thread returns earlier
+        pair_finish<uint16_t>(fix, M, keep, info);
+    }
 }
 
 // ------------------------------------------------------------------ host side
@@ -504,7 +560,16 @@ constexpr LdgShape ldg_shape(int bits, int group, int nb) {
 struct LdgPlan {
     int64_t total_units = 0, total_tiles = 0, total_warps = 0;
     int grid = 1, maxc = 2;
+    bool pair = false;
 };
+
+// Pair mode: clusters of two CTAs that each get a whole number of tiles, so that no tile
+// is shared outside a cluster and no GPU-scope ticket is left at the end of the launch;
+// chosen for the 16-warp shapes when the grid is full and the largest pair has at most
+// kPairSlack more units than the average.  (On the 8-warp shapes the pair barrier cost
+// more than the tickets it saves.)
+constexpr bool kLdgPairMode = true;
+constexpr double kPairSlack = 0.06;
 
 static LdgPlan plan_ldg(const int64_t* n, const int64_t* k, int count, int nw) {
     LdgPlan pl;
@@ -527,6 +592,26 @@ static LdgPlan plan_ldg(const int64_t* n, const int64_t* k, int count, int nw) {
     // warps that share one tile: the slices are floor(w S / W), so a window of ksb units
     // meets at most ceil(ksb W / S) + 1 of them; one more slot of margin
     pl.maxc = (int)(ceil_div(max_ksb * pl.total_warps, std::max<int64_t>(pl.total_units, 1)) + 2);
+    const int64_t P = sm_count() / 2;
+    if (kLdgPairMode && nw == 16 && P >= 1 && pl.grid == sm_count() && pl.total_tiles >= P) {
+        auto first_unit = [&](int64_t T) {
+            int64_t u = 0;
+            for (int i = 0; i < count; i++) {
+                const int64_t nt = n[i] / 16, ksb = k[i] / kLdgChunk;
+                if (T < nt) return u + T * ksb;
+                T -= nt;
+                u += nt * ksb;
+            }
+            return u;
+        };
+        int64_t worst = 0;
+        for (int64_t p = 0; p < P; p++)
+            worst = std::max(worst, first_unit((p + 1) * pl.total_tiles / P) - first_unit(p * pl.total_tiles / P));
+        if ((double)worst * (double)P <= (1.0 + kPairSlack) * (double)pl.total_units) {
+            pl.pair = true;
+            pl.grid = (int)(2 * P);
+        }
+    }
     return pl;
 }
 
@@ -569,13 +654,13 @@ static lbq_status launch_ldg_inst(int grid, bool smemp, bool bf16, int smem, cud
             constexpr auto kh = k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.NW, true, false>;
             const lbq_status s = bf16 ? ldg_smem_attr<kb>(kLdgSmemBudget) : ldg_smem_attr<kh>(kLdgSmemBudget);
             if (s != LBQ_OK) return s;
-            return launch_pdl(bf16 ? kb : kh, grid, sh.NW * 32, (size_t)smem, st, args, prep);
+            return launch_pdl_cluster(bf16 ? kb : kh, grid, args.pair ? 2 : 1, sh.NW * 32, (size_t)smem, st, args, prep);
         }
     }
     constexpr auto kg = k_gemv_group_ldg<B, GROUP, NB, sh.D, sh.NW, false, false>;
     const lbq_status s = ldg_smem_attr<kg>(kLdgSmemBudget);
     if (s != LBQ_OK) return s;
-    return launch_pdl(kg, grid, sh.NW * 32, (size_t)smem, st, args, prep);
+    return launch_pdl_cluster(kg, grid, args.pair ? 2 : 1, sh.NW * 32, (size_t)smem, st, args, prep);
 }
 
 template <int B, int GROUP>
@@ -662,6 +747,8 @@ lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count,
     prep.M = (int)M;
     args.total_units = pl.total_units;
     args.total_warps = pl.total_warps;
+    args.total_tiles = pl.total_tiles;
+    args.pair = pl.pair ? 1 : 0;
     args.count = count;
     args.M = (int)M;
     args.maxc = pl.maxc;
@@ -669,7 +756,7 @@ lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count,
     // prepared activations in each CTA's shared memory when they fit, else one prep launch;
     // the scale/zero rings follow them (or start the shared memory)
     const int ring = shape.NW * kScaleRing * scale_slot_bytes(group);
-    const int fixb = al16(shape.NW * 2 * 16 * M * 4 + shape.NW * 2 * 4);
+    const int fixb = al16((int64_t)cta_fix_bytes(shape.NW, (int)M));
     const bool smemp = NB == 1 && soff + ring + 256 + fixb <= kLdgSmemBudget;
     args.sring = smemp ? al16(soff) : 0;
     args.szero = args.sring + ring;

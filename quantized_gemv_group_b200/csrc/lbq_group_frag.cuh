@@ -116,20 +116,31 @@ __device__ __forceinline__ void tile_epilogue_any(const float (&acc)[NB][2], boo
 // that lies inside the CTA's range is stored at once; one shared with other CTAs goes
 // through the global ticket (the last of its CTAs adds the CTA sums in CTA order), so at
 // most two tiles per CTA pay for a GPU-scope atomic, and the sum order is fixed.
+//
+// Pair mode (clusters of two CTAs, each pair given a whole number of tiles) has no
+// GPU-scope ticket: the one tile the pair's two CTAs share is finished by rank 0, which
+// receives rank 1's sum in its shared memory (recv) across the cluster barrier.
 struct CtaFix {
     float* val;     // [NW][2][16 * M] partial sums, element tok * 16 + row
     int* tile;      // [NW][2] tile index of each slot, -1 if unused
+    float* recv;    // [16 * M] pair mode: rank 1's sum of the shared tile (in rank 0)
 };
 
-__device__ __forceinline__ size_t cta_fix_bytes(int nw, int M) {
-    return (size_t)nw * 2 * 16 * M * 4 + (size_t)nw * 2 * 4;
+__host__ __device__ __forceinline__ size_t cta_fix_bytes(int nw, int M) {
+    return (size_t)nw * 2 * 16 * M * 4 + (size_t)nw * 2 * 4 + (size_t)16 * M * 4;
 }
 __device__ __forceinline__ CtaFix cta_fix_at(uint8_t* base, int nw, int M) {
     CtaFix f;
     f.val = reinterpret_cast<float*>(base);
-    f.tile = reinterpret_cast<int*>(base + (size_t)nw * 2 * 16 * M * 4);
+    f.recv = reinterpret_cast<float*>(base + (size_t)nw * 2 * 16 * M * 4);
+    f.tile = reinterpret_cast<int*>(base + (size_t)nw * 2 * 16 * M * 4 + (size_t)16 * M * 4);
     return f;
 }
+// Rank 0's share of the pair's shared tile, kept in registers across the cluster barrier.
+struct PairKeep {
+    int T = -1;
+    float v[8];     // elements lane, lane + 32, ... (16 * M <= 256)
+};
 __device__ __forceinline__ void cta_fix_clear(const CtaFix& f, int warp, int lane) {
     if (lane < 2) f.tile[warp * 2 + lane] = -1;
 }
@@ -169,11 +180,13 @@ __device__ __forceinline__ void tile_store_full(const float (&acc)[NB][2], int M
 // output rows y[tok * n + row0 + 0..15].  The launch's W warps split S units evenly
 // (warp w: [w S / W, (w + 1) S / W)), NW per CTA; u_begin is this warp's first unit,
 // [C0, C1) the CTA's range and cta its index.
+// pair: 0 = tickets, 1 = pair mode in rank 0 (the shared tile goes to keep), 2 = pair mode
+// in rank 1 (the shared tile's sum is stored into rank 0's recv).
 template <class Y, class Info>
 __device__ __forceinline__ void cta_fix_finish(const CtaFix& f, int NW, int warp, int M, int64_t u_begin, int64_t C0,
                                                int64_t C1, int64_t S, int64_t W, int64_t cta,
                                                float* __restrict__ partials, unsigned* __restrict__ counters, int maxc,
-                                               Info info) {
+                                               Info info, int pair = 0, PairKeep* keep = nullptr) {
     const int lane = threadIdx.x & 31;
     const int E = 16 * M;
 #pragma unroll 1
@@ -187,6 +200,21 @@ __device__ __forceinline__ void cta_fix_finish(const CtaFix& f, int NW, int warp
         int w_end = warp + 1;
         while (w_end < NW && f.tile[w_end * 2] == T) w_end++;
         const bool inside = first_u >= C0 && first_u + units <= C1;
+        if (!inside && pair != 0) {
+            const uint32_t rr = pair == 2 ? cluster_map_smem(smem_u32(f.recv), 0) : 0u;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int e = lane + 32 * j;
+                if (e < E) {
+                    float s = f.val[(warp * 2 + k) * E + e];
+                    for (int w2 = warp + 1; w2 < w_end; w2++) s += f.val[(w2 * 2) * E + e];
+                    if (pair == 2) st_cluster_f32(rr + 4u * (uint32_t)e, s);
+                    else keep->v[j] = s;
+                }
+            }
+            if (pair == 1) keep->T = T;
+            continue;
+        }
         int64_t cf = 0, count = 1;
         float* p0 = nullptr;
         if (!inside) {
@@ -225,6 +253,21 @@ __device__ __forceinline__ void cta_fix_finish(const CtaFix& f, int NW, int warp
             __syncwarp();
             if (lane == 0) counters[T] = 0u;
         }
+    }
+}
+
+// Pair mode, after the cluster barrier: rank 0 adds rank 1's sum and stores the shared tile.
+template <class Y, class Info>
+__device__ __forceinline__ void pair_finish(const CtaFix& f, int M, const PairKeep& keep, Info info) {
+    if (keep.T < 0) return;
+    const int lane = threadIdx.x & 31;
+    int64_t first_u, units, n, row0;
+    Y* y;
+    info(keep.T, first_u, units, y, n, row0);
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        const int e = lane + 32 * j;
+        if (e < 16 * M) store_out(y + (int64_t)(e / 16) * n + row0 + (e % 16), keep.v[j] + f.recv[e]);
     }
 }
 

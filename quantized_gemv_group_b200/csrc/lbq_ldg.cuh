@@ -96,20 +96,35 @@ __device__ __forceinline__ PrepOut prep_quantize8(const float (&v)[8], int E) {
 
 // ------------------------------------------------------------------ host side
 
+// Programmatic-dependent launch; cluster > 1 groups the CTAs into thread-block clusters of
+// that many (grid a multiple of it).
 template <class Kern, class... Args>
-inline lbq_status launch_pdl(Kern kern, int grid, int threads, size_t smem, cudaStream_t st, const Args&... args) {
+inline lbq_status launch_pdl_cluster(Kern kern, int grid, int cluster, int threads, size_t smem, cudaStream_t st,
+                                     const Args&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    int na = 1;
+    if (cluster > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = (unsigned)cluster;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        na = 2;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = na;
     if (cudaLaunchKernelEx(&cfg, kern, args...) != cudaSuccess) return LBQ_ERR_CUDA;
     return launch_status();
+}
+template <class Kern, class... Args>
+inline lbq_status launch_pdl(Kern kern, int grid, int threads, size_t smem, cudaStream_t st, const Args&... args) {
+    return launch_pdl_cluster(kern, grid, 1, threads, smem, st, args...);
 }
 
 template <auto KERN>
