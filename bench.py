@@ -48,7 +48,7 @@ FALLBACK_HBM_GBS = 6650.0
 # the step's launches), from the ncu capture summarised in
 # profiles/k_gemv_group_ldg__llama2_70b_block_int4_g64_m1.md (None: not captured for the
 # current kernel version).
-NCU_TRAFFIC = {"block": (481.64e6 + 0.54e6) / 4, "sweep80": None, "binlr": None}
+NCU_TRAFFIC = {"block": (481.717e6 + 0.270e6) / 4, "sweep80": None, "binlr": None}
 
 
 # ---------------------------------------------------------------- helpers
