@@ -222,6 +222,10 @@ __global__ void __launch_bounds__(NW * 32, 1)
     constexpr int PF = 16384 / (512 * B);
     extern __shared__ __align__(16) uint8_t smem[];
     griddep_launch_dependents();
+    // pair mode: the two CTAs prepare half of the activations each, into both shared
+    // memories; the partner must have started before the first remote store
+    const bool pairp = SMEMP && a.pair != 0;
+    if (pairp) cluster_arrive_relaxed();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
@@ -326,14 +330,20 @@ __global__ void __launch_bounds__(NW * 32, 1)
     }
     griddep_wait();
     if constexpr (SMEMP) {
-        // this CTA's copy of the prepared activations: warp w takes chunks w, w + 8, ...
-        // of every token of every slot, rotated by the CTA index so that the CTAs do not all
-        // read the same lines of x at once (no divisions on the way)
+        // this CTA's copy of the prepared activations: warp w takes chunks w, w + NW, ...
+        // of every token of every slot (in pair mode the pair's 2 NW warps split them and
+        // each chunk is stored into both CTAs), rotated by the CTA (pair) index so that the
+        // CTAs do not all read the same lines of x at once (no divisions on the way)
+        if (pairp) cluster_wait();
+        const uint32_t peer = (blockIdx.x & 1) ^ 1u;
+        const int pw = pairp ? 2 * NW : NW;
+        const int pwi = pairp ? (int)(blockIdx.x & 1) * NW + warp : warp;
+        const unsigned pidx = pairp ? blockIdx.x >> 1 : blockIdx.x;
         for (int si = 0; si < pa.count; si++) {
             const PrepSlot& Q = pa.s[si];
             const int kch = (int)(Q.k / kLdgChunk);
             const int k32 = (int)Q.k;
-            const int rot = (int)(blockIdx.x % (unsigned)kch);
+            const int rot = (int)(pidx % (unsigned)kch);
             for (int m = 0; m < M; m++) {
                 const uint16_t* xm = Q.x + (int64_t)m * k32;
                 int8_t* row_h = reinterpret_cast<int8_t*>(smem + Q.sp) + (int64_t)(2 * m) * k32;
@@ -341,32 +351,42 @@ __global__ void __launch_bounds__(NW * 32, 1)
                 int* ex = reinterpret_cast<int*>(smem + Q.se) + m * kch;
                 // a warp's chunks are independent: issue kPrepBatch loads of x together
                 constexpr int PB = kPrepBatch;
-                for (int cw0 = warp; cw0 < kch; cw0 += NW * PB) {
+                for (int cw0 = pwi; cw0 < kch; cw0 += pw * PB) {
                     uint4 raw[PB];
 #pragma unroll
                     for (int j = 0; j < PB; j++) {
-                        const int cw = cw0 + j * NW;
+                        const int cw = cw0 + j * pw;
                         const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
                         if (cw < kch) raw[j] = prep_load(xm + ch * kLdgChunk, lane);
                     }
 #pragma unroll
                     for (int j = 0; j < PB; j++) {
-                        const int cw = cw0 + j * NW;
+                        const int cw = cw0 + j * pw;
                         if (cw < kch) {
                             const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
                             const PrepOut r = prep_convert<GROUP, BF16>(raw[j]);
-                            *reinterpret_cast<uint2*>(row_h + ch * kLdgChunk + plane_off(lane)) = r.hi;
-                            *reinterpret_cast<uint2*>(row_h + k32 + ch * kLdgChunk + plane_off(lane)) = r.lo;
+                            int8_t* ph = row_h + ch * kLdgChunk + plane_off(lane);
+                            *reinterpret_cast<uint2*>(ph) = r.hi;
+                            *reinterpret_cast<uint2*>(ph + k32) = r.lo;
                             constexpr int LPG = GROUP / 8;
-                            if (lane % LPG == 0) xs[ch * (kLdgChunk / GROUP) + lane / LPG] = (float)r.gsum;
+                            float* px = xs + ch * (kLdgChunk / GROUP) + lane / LPG;
+                            if (lane % LPG == 0) *px = (float)r.gsum;
                             if (lane == 0) ex[ch] = r.E;
+                            if (pairp) {
+                                st_cluster_u32x2(cluster_map_smem(smem_u32(ph), peer), r.hi);
+                                st_cluster_u32x2(cluster_map_smem(smem_u32(ph + k32), peer), r.lo);
+                                if (lane % LPG == 0)
+                                    st_cluster_f32(cluster_map_smem(smem_u32(px), peer), (float)r.gsum);
+                                if (lane == 0) st_cluster_s32(cluster_map_smem(smem_u32(ex + ch), peer), r.E);
+                            }
                         }
                     }
                 }
             }
         }
     }
-    __syncthreads();
+    if (pairp) cluster_sync_all();        // both halves of the activations are in place
+    else __syncthreads();
 #pragma unroll
     for (int d = 0; d < D; d++)
         if (u_begin + d < u_end) load_next(wb[d]);

@@ -419,6 +419,36 @@ def test_block_linears_int4_g64_sampled(lin):
     assert _rel(_np(y.float())[:, rows], ref) <= REL_TOL
 
 
+@pytest.mark.parametrize("M", [1, 3])
+@pytest.mark.parametrize("bits,group", [(4, 64), (5, 32)], ids=["int4_g64_pairs", "int5_g32_tickets"])
+def test_gemv_group_multi_qkv_full_grid_sampled(bits, group, M):
+    """The grouped q/k/v launch at 70B shapes fills the grid: 16-warp shapes run as pairs of
+    CTAs whose shared tile is finished across the cluster barrier, 8-warp shapes finish
+    CTA-crossing tiles by ticket.  Sampled rows of every product match the oracle and a
+    second launch gives the same bits."""
+    shapes = [(8192, 8192), (1024, 8192), (1024, 8192)]
+    x = synth.activations(M, 8192, seed=31, device=DEV)
+    probs, rows_l, ref_l = [], [], []
+    for i, (n, k) in enumerate(shapes):
+        W = synth.weight(n, k, seed=300 + i, device=DEV)
+        codes, s, z = lbq.lbq_quantize_rtn(W, bits, group)
+        del W
+        packed = lbq.lbq_pack(codes, bits)
+        y = torch.full((M, n), float("nan"), dtype=torch.float16, device=DEV)
+        probs.append((x, packed, s, z, y, n, k))
+        rows = _sample_rows(n, 24, 40 + i)
+        rows_l.append(rows)
+        ref_l.append(orc.gemv_group(_u16(x), _np(packed), _u16(s), _u16(z), n, k, bits, group,
+                                    layout=orc.LAYOUT_KERNEL, rows=rows))
+    lbq.lbq_gemv_group_multi(probs, bits, group)
+    first = [pr[4].clone() for pr in probs]
+    lbq.lbq_gemv_group_multi(probs, bits, group)
+    for pr, y1, rows, ref in zip(probs, first, rows_l, ref_l):
+        assert torch.equal(pr[4], y1)
+        assert not torch.isnan(pr[4].float()).any()
+        assert _rel(_np(pr[4].float())[:, rows], ref) <= REL_TOL
+
+
 @pytest.mark.parametrize("shape", [(28672, 8192), (8192, 28672)], ids=["gate_up", "down"])
 @pytest.mark.parametrize("M", [4, 16])
 def test_prefill_shapes_int4_g128_bf16_sampled(shape, M):
