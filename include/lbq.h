@@ -202,8 +202,8 @@ lbq_status lbq_gemm_group(const void* x, lbq_dtype x_dtype, int64_t M,
  * (canonical: u32 words, bit 1 = +1).  s1 [d_out], s2 [d_in] f16.
  * x: [M x d_in] in x_dtype, y: [M x d_out] f16.  r % 32 == 0, d_in % 32 == 0.
  * The LBQ_LAYOUT_KERNEL path converts s2 ⊙ x and the intermediate t to 16-bit
- * fixed point with one power-of-two scale per token and stage (integer tensor
- * cores, exact int32 sums); relative error of y stays below 1e-3.
+ * fixed point with one power-of-two scale per token and 256-column chunk (integer
+ * tensor cores, exact int32 sums per chunk); relative error of y stays below 1e-3.
  * ws: lbq_workspace_bytes(LBQ_OP_GEMV_BINLR, M, d_out, d_in, r) bytes. */
 lbq_status lbq_gemv_binlr(const void* x, lbq_dtype x_dtype, int64_t M,
                           const void* U, const void* Vt, const void* s1, const void* s2,
