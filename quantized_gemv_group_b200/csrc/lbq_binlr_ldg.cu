@@ -46,6 +46,7 @@ struct BinStageArgs {
     int M, maxc;
     int sp, sv, se, szero;      // shared-memory offsets: planes, chunk sums, exponents, zero chunk,
     int sfix;                   // CTA-level tile finish (CtaFix)
+    int cluster2;               // 1: clusters of two CTAs that share the input prep
 };
 
 // Byte offset, in a 256-column chunk of a plane row, of column 32p + 16h + 4c + j: the
@@ -124,6 +125,10 @@ __global__ void __launch_bounds__(NW * 32, 1) k_binlr_ldg(const __grid_constant_
     constexpr int PF = 16;                     // units prefetched into L2 before the wait
     extern __shared__ __align__(16) uint8_t smem[];
     griddep_launch_dependents();
+    // clusters of two: each CTA prepares half of the stage input, into both shared
+    // memories; the partner must have started before the first remote store
+    const bool c2 = a.cluster2 != 0;
+    if (c2) cluster_arrive_relaxed();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
@@ -160,19 +165,23 @@ __global__ void __launch_bounds__(NW * 32, 1) k_binlr_ldg(const __grid_constant_
     griddep_wait();
 
     // ---- prepare the stage input in one pass: per 256-column chunk one power-of-two scale,
-    // the int8 planes and the exact chunk sum; the chunk order is rotated by the CTA index
-    // so that the CTAs do not all read the same lines at once
+    // the int8 planes and the exact chunk sum; the chunk order is rotated by the CTA (pair)
+    // index so that the CTAs do not all read the same lines at once
+    if (c2) cluster_wait();
+    const uint32_t peer = (blockIdx.x & 1) ^ 1u;
+    const int pw = c2 ? 2 * NW : NW;                                // warps sharing the prep
+    const int pwi = c2 ? (int)(blockIdx.x & 1) * NW + warp : warp;
     const int kch = (int)(a.cpad / kLdgChunk);
     const int ntask = M * kch;                   // (token, chunk) pairs
-    const int rot = (int)(blockIdx.x % (unsigned)kch);
+    const int rot = (int)((c2 ? blockIdx.x >> 1 : blockIdx.x) % (unsigned)kch);
     int* expo = reinterpret_cast<int*>(smem + a.se);
     int* vsum = reinterpret_cast<int*>(smem + a.sv);
     // a warp's chunks are independent: issue the loads of kBinPrepBatch of them together
-    for (int t0 = warp; t0 < ntask; t0 += NW * kBinPrepBatch) {
+    for (int t0 = pwi; t0 < ntask; t0 += pw * kBinPrepBatch) {
         uint4 r0[kBinPrepBatch], r1[kBinPrepBatch];
 #pragma unroll
         for (int j = 0; j < kBinPrepBatch; j++) {
-            const int t = t0 + j * NW;
+            const int t = t0 + j * pw;
             if (t < ntask) {
                 const int m = t / kch, cw = t - m * kch;
                 const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
@@ -181,7 +190,7 @@ __global__ void __launch_bounds__(NW * 32, 1) k_binlr_ldg(const __grid_constant_
         }
 #pragma unroll
         for (int j = 0; j < kBinPrepBatch; j++) {
-            const int t = t0 + j * NW;
+            const int t = t0 + j * pw;
             if (t < ntask) {
                 const int m = t / kch, cw = t - m * kch;
                 const int ch = cw + rot < kch ? cw + rot : cw + rot - kch;
@@ -191,18 +200,29 @@ __global__ void __launch_bounds__(NW * 32, 1) k_binlr_ldg(const __grid_constant_
                 // elements 8 lane + 0..3 and + 4..7: columns 32p + 16h + 4c' + j
                 const int p = lane >> 2, h = (lane & 3) >> 1, c0 = 2 * (lane & 1);
                 int8_t* base = reinterpret_cast<int8_t*>(smem + a.sp) + (int64_t)(2 * m) * a.cpad + ch * kLdgChunk;
-                *reinterpret_cast<uint32_t*>(base + bin_plane_off(p, h, c0)) = r.hi.x;
-                *reinterpret_cast<uint32_t*>(base + bin_plane_off(p, h, c0 + 1)) = r.hi.y;
-                *reinterpret_cast<uint32_t*>(base + a.cpad + bin_plane_off(p, h, c0)) = r.lo.x;
-                *reinterpret_cast<uint32_t*>(base + a.cpad + bin_plane_off(p, h, c0 + 1)) = r.lo.y;
+                uint32_t* q[4] = {reinterpret_cast<uint32_t*>(base + bin_plane_off(p, h, c0)),
+                                  reinterpret_cast<uint32_t*>(base + bin_plane_off(p, h, c0 + 1)),
+                                  reinterpret_cast<uint32_t*>(base + a.cpad + bin_plane_off(p, h, c0)),
+                                  reinterpret_cast<uint32_t*>(base + a.cpad + bin_plane_off(p, h, c0 + 1))};
+                const uint32_t qv[4] = {r.hi.x, r.hi.y, r.lo.x, r.lo.y};
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    *q[i] = qv[i];
+                    if (c2) st_cluster_s32(cluster_map_smem(smem_u32(q[i]), peer), (int)qv[i]);
+                }
                 if (lane == 0) {
                     vsum[m * kch + ch] = r.gsum;
                     expo[m * kch + ch] = r.E;
+                    if (c2) {
+                        st_cluster_s32(cluster_map_smem(smem_u32(vsum + m * kch + ch), peer), r.gsum);
+                        st_cluster_s32(cluster_map_smem(smem_u32(expo + m * kch + ch), peer), r.E);
+                    }
                 }
             }
         }
     }
-    __syncthreads();
+    if (c2) cluster_sync_all();                  // both halves of the input are in place
+    else __syncthreads();
     const CtaFix fix = cta_fix_at(smem + a.sfix, NW, M);
     cta_fix_clear(fix, warp, lane);
     const int head_tile = ct;
@@ -313,12 +333,16 @@ struct BinLdgPlan {
 // Warps per CTA and register ring depth of the sign stream (one CTA per SM: the stage
 // input is prepared once per SM).
 constexpr int kBinNW = 16, kBinD = 8;
+// Launches of at least this many CTAs run as clusters of two that prepare half of the
+// stage input each (the prep is latency-bound: a 28672-wide input costs ~7 us per CTA).
+constexpr int kBinClusterMinGrid = 32;
 
 static void bin_stage_plan(int64_t rows, int64_t cpad, int64_t& units, int64_t& warps, int& grid, int& maxc) {
     const int64_t ksb = cpad / kLdgChunk;
     units = rows / 16 * ksb;
     constexpr int64_t kMinUnitsPerWarp = 4;
     grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sm_count(), ceil_div(units, kBinNW * kMinUnitsPerWarp)));
+    if (grid >= kBinClusterMinGrid) grid &= ~1;    // clusters of two share the input prep
     warps = std::min<int64_t>((int64_t)grid * kBinNW, std::max<int64_t>(units, 1));
     maxc = (int)(ceil_div(ksb * warps, std::max<int64_t>(units, 1)) + 2);
 }
@@ -358,7 +382,7 @@ static lbq_status launch_bin_stage(const BinStageArgs& a, int grid, int smem, cu
     constexpr auto kern = k_binlr_ldg<STAGE2, kBinD, kBinNW, BF16>;
     const lbq_status s = ldg_smem_attr<kern>(200 * 1024);
     if (s != LBQ_OK) return s;
-    return launch_pdl(kern, grid, kBinNW * 32, (size_t)smem, st, a);
+    return launch_pdl_cluster(kern, grid, a.cluster2 ? 2 : 1, kBinNW * 32, (size_t)smem, st, a);
 }
 
 lbq_status launch_gemv_binlr_ldg(const void* x, bool bf16, int64_t M, const void* U, const void* Vt, const void* s1,
@@ -398,6 +422,7 @@ lbq_status launch_gemv_binlr_ldg(const void* x, bool bf16, int64_t M, const void
         a.sfix = a.szero + 256;
         const int smem = bin_smem_bytes(M, a.cpad);
         const int grid = st2 ? pl.grid2 : pl.grid1;
+        a.cluster2 = grid >= kBinClusterMinGrid ? 1 : 0;
         lbq_status s;
         if (st2) s = bf16 ? launch_bin_stage<true, true>(a, grid, smem, st) : launch_bin_stage<true, false>(a, grid, smem, st);
         else s = bf16 ? launch_bin_stage<false, true>(a, grid, smem, st) : launch_bin_stage<false, false>(a, grid, smem, st);
