@@ -45,10 +45,11 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the step's kernel (mean over
-# the step's launches), from the ncu capture summarised in
-# profiles/k_gemv_group_ldg__llama2_70b_block_int4_g64_m1.md (None: not captured for the
-# current kernel version).
-NCU_TRAFFIC = {"block": (481.717e6 + 0.270e6) / 4, "sweep80": None, "binlr": None}
+# the step's launches), from the ncu captures summarised in
+# profiles/k_gemv_group_ldg__llama2_70b_block_int4_g64_m1.md and
+# profiles/k_binlr_ldg__gate_shape_r5088_m1.md (None: not captured for the current kernel
+# version).
+NCU_TRAFFIC = {"block": (481.705e6 + 0.314e6) / 4, "sweep80": None, "binlr": 55.545e6 / 8}
 
 
 # ---------------------------------------------------------------- helpers
