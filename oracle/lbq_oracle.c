@@ -23,7 +23,7 @@
  *    (nramos.dev), section "1. NanoQuant — sub-1-bit PTQ", bullet
  *    "Formulación": W ≈ s1 ⊙ (U±1 · V±1ᵀ) ⊙ s2ᵀ with binary low-rank U, V.
  *
- * Readings where the pages are silent (all listed in the design doc):
+ * Readings where the pages are silent:
  *  R1  the group offset is an integer zero-point z with w_hat = s*(q - z);
  *      the grid range is forced to contain 0, so z lies in [0, 2^b-1];
  *  R2  the fp32 scale is rounded UP to fp16, so (hi-lo)/s <= 2^b-1 and
@@ -38,7 +38,7 @@
  *  R8  the fragment-interleaved kernel layout is a permutation of the same
  *      bits (tiles of 16 rows x 256 columns in integer tensor-core fragment
  *      order); its index map is written out in orc_kernel_pos() below from
- *      the specification in DESIGN.md ("Kernel layout"), independently of the
+ *      the written specification restated above it, independently of the
  *      CUDA packer.
  *
  * Parity pins for every function live in tests/test_oracle_*.py; there is
@@ -227,7 +227,7 @@ int orc_unpack_canonical(const uint8_t* in, int64_t n, int64_t k, int bits, uint
 /* ------------------------------------------------------------------------- */
 /* Kernel (fragment-interleaved) layout for group codes (reading R8).         */
 /*                                                                            */
-/* Specification, restated from DESIGN.md "Kernel layout":                    */
+/* Specification of the layout:                                             */
 /*  * a b-bit code is split into a low plane of width w0 and a high plane    */
 /*    of width w1 = b - w0: b=2 -> (2), b=3 -> (2,1), b=4 -> (4),              */
 /*    b=5 -> (4,1), b=6 -> (4,2).  Low plane value = q mod 2^w0, high plane   */
@@ -526,7 +526,7 @@ int orc_pack_signs(const int8_t* pm1, int64_t rows, int64_t cols, uint32_t* out)
 /* ------------------------------------------------------------------------- */
 /* Kernel (fragment-interleaved) layout for sign matrices (reading R8).       */
 /*                                                                            */
-/* Specification, restated from DESIGN.md "Kernel layout, signs": a sign      */
+/* Specification of the layout: a sign                                      */
 /* matrix [rows x cols] (rows % 16 == 0) has its columns padded with bit 0   */
 /* up to cols_pad = 256*ceil(cols/256).  Tile T (16 rows) and superblock S    */
 /* (256 columns) occupy 512 bytes at byte offset (T*(cols_pad/256) + S)*512.  */
