@@ -354,49 +354,79 @@ WORKLOADS = {"block": BlockWorkload, "sweep80": Sweep80Workload, "binlr": BinlrW
 
 
 # ---------------------------------------------------------------- CPU oracle legs
-def _oracle_block_sample(wk, frac_rows, check=True):
-    """Oracle GEMV on a sample of output rows of copy 0 of every linear.
-    Returns (bytes of the sampled work, seconds, worst rel-L2 of the GPU result)."""
+def _oracle_block_inputs(dev, stride):
+    """Inputs of the oracle's sampled block GEMV, made by the oracle itself on the host: the
+    seeded synthetic weights of copy 0 of every block linear (only every `stride`-th 16-row
+    tile), quantized and packed by oracle/, and the seeded activations of its launch group.
+    One row of each sampled tile is the sample: 1/(16 stride) of the output rows."""
+    import oracle as orc
+    out = []
+    for p, l in enumerate(wl.block_linears()):
+        n, k = l.d_out, l.d_in
+        gi = next(i for i, grp in enumerate(BlockWorkload.LAUNCHES) if l.name in grp)
+        x = synth.activations(1, k, seed=900 + gi, device=dev)
+        W = synth.weight(n, k, seed=synth.tensor_seed(0, p), device=dev)
+        tiles = np.arange(0, n // 16, stride)
+        idx = (tiles[:, None] * 16 + np.arange(16)[None, :]).reshape(-1)
+        w_sub = synth.bits_u16(W[torch.from_numpy(idx).to(W.device)])
+        del W
+        codes, s_, z_ = orc.quantize_rtn(w_sub, BlockWorkload.bits, BlockWorkload.group)
+        packed = orc.pack(codes, BlockWorkload.bits, layout=orc.LAYOUT_KERNEL)
+        pick = np.arange(len(tiles)) % 16                      # the sampled row of each tile
+        out.append({"p": p, "n_sub": len(idx), "k": k, "xh": synth.bits_u16(x), "packed": packed, "s": s_,
+                    "z": z_, "rows": np.arange(len(tiles)) * 16 + pick, "rows_global": tiles * 16 + pick})
+    return out
+
+
+def _oracle_block_run(inputs, wk=None):
+    """Oracle GEMV on the prepared samples: (algorithmic bytes of the sampled work, seconds,
+    worst rel-L2 of the GPU outputs of copy 0 at the same rows if wk is given)."""
     import oracle as orc
     tot_bytes, tot_s, worst = 0, 0.0, 0.0
-    for p, l in enumerate(wk.linears):
-        packed, s, z, _ = wk.sets[0][p]
-        n, k = l.d_out, l.d_in
-        rows = np.arange(0, n, max(1, int(round(1 / frac_rows))), dtype=np.int64)
-        ph, sh, zh = packed.cpu().numpy(), synth.bits_u16(s), synth.bits_u16(z)
-        xh = synth.bits_u16(wk.x[p])
+    bits, group = BlockWorkload.bits, BlockWorkload.group
+    for d in inputs:
         t0 = time.perf_counter()
-        ref = orc.gemv_group(xh, ph, sh, zh, n, k, wk.bits, wk.group, layout=orc.LAYOUT_KERNEL, rows=rows)
+        ref = orc.gemv_group(d["xh"], d["packed"], d["s"], d["z"], d["n_sub"], d["k"], bits, group,
+                             layout=orc.LAYOUT_KERNEL, rows=d["rows"])
         tot_s += time.perf_counter() - t0
-        tot_bytes += wl.gemv_algorithmic_bytes(len(rows), k, wk.bits, wk.group, 1)
-        if check:
-            worst = max(worst, orc.rel_l2(wk.y[p].float().cpu().numpy()[:, rows], ref))
+        tot_bytes += wl.gemv_algorithmic_bytes(len(d["rows"]), d["k"], bits, group, 1)
+        if wk is not None:
+            worst = max(worst, orc.rel_l2(wk.y[d["p"]].float().cpu().numpy()[:, d["rows_global"]], ref))
     return tot_bytes, tot_s, worst
 
 
+def _block_config():
+    """The block workload's config dict, without building the workload."""
+    from types import SimpleNamespace
+    return BlockWorkload.config(SimpleNamespace(linears=wl.block_linears(), bits=BlockWorkload.bits,
+                                                group=BlockWorkload.group, LAUNCHES=BlockWorkload.LAUNCHES,
+                                                M=1, copies=BlockWorkload.copies))
+
+
 def run_reference(args, dev):
-    """--impl reference: the CPU oracle on a bounded sample of the block workload."""
+    """--impl reference: the CPU oracle on a bounded sample of the block workload, on inputs
+    the oracle quantizes and packs itself (no GPU code on this arm)."""
     import oracle as orc
     ws, rank, _ = _rank_info()
     if rank != 0:
         return
-    wk = BlockWorkload(dev) if torch.cuda.is_available() else None
-    frac = 1.0 / 128
+    stride = 8
+    inputs = _oracle_block_inputs(dev, stride)
     cores = orc.num_threads()
     for _ in range(args.warmup):
-        _oracle_block_sample(wk, frac, check=False)
+        _oracle_block_run(inputs)
     secs, byts = [], 0
     for _ in range(args.steps):
-        b, s, _ = _oracle_block_sample(wk, frac, check=False)
+        b, s, _ = _oracle_block_run(inputs)
         secs.append(s)
         byts = b
     total = sum(secs)
     value = byts * args.steps / total / 1e9
-    sample = f"1/{int(1/frac)} of the output rows of each of the 7 block linears per step"
+    sample = f"1/{16 * stride} of the output rows of each of the 7 block linears per step"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": wk.config(),
+            "data": "synthetic", "config": _block_config(),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -530,8 +560,7 @@ def run_gpu(args, dev):
         with torch.cuda.stream(stream):
             wk.run_copy(0)                # outputs of copy 0, the one the oracle samples
         torch.cuda.synchronize()
-        frac = 1.0 / 64
-        b, s, worst = _oracle_block_sample(wk, frac, check=True)
+        b, s, worst = _oracle_block_run(_oracle_block_inputs(dev, 4), wk)
         line["cpu_baseline"] = {"value": b / s / 1e9, "unit": UNIT, "cores": orc.num_threads(), "kind": "oracle",
                                 "sample": "1/64 of the output rows of each of the 7 block linears (copy 0)"}
         line["parity_sampled_rel_l2"] = worst
