@@ -137,7 +137,10 @@ size_t lbq_workspace_bytes(lbq_op op, int64_t M, int64_t n, int64_t k, int64_t r
  * activation type).  packed in `layout` (lbq_pack),
  * scales/zeros [n x k/group] f16 as written by lbq_quantize_rtn.  x, packed,
  * scales, zeros 16-byte aligned (LBQ_LAYOUT_KERNEL) or 4-byte (canonical).
- * ws: lbq_workspace_bytes(LBQ_OP_GEMV_GROUP, M, n, k, 0) bytes. */
+ * ws: lbq_workspace_bytes(LBQ_OP_GEMV_GROUP, M, n, k, 0) bytes.
+ * Launches of the kernel layout use one CTA per SM and, when they fill the GPU, may run
+ * as thread-block clusters of two CTAs (no CTA of a launch waits for another cluster).
+ * Results are deterministic: every split sum is added in a fixed order. */
 lbq_status lbq_gemv_group(const void* x, lbq_dtype x_dtype, int64_t M,
                           const void* packed, const void* scales, const void* zeros,
                           int64_t n, int64_t k, int bits, int group, lbq_layout layout,
