@@ -354,14 +354,17 @@ WORKLOADS = {"block": BlockWorkload, "sweep80": Sweep80Workload, "binlr": BinlrW
 
 
 # ---------------------------------------------------------------- CPU oracle legs
-def _oracle_block_inputs(dev, stride):
+def _oracle_block_inputs(dev, stride, only=None):
     """Inputs of the oracle's sampled block GEMV, made by the oracle itself on the host: the
     seeded synthetic weights of copy 0 of every block linear (only every `stride`-th 16-row
     tile), quantized and packed by oracle/, and the seeded activations of its launch group.
-    One row of each sampled tile is the sample: 1/(16 stride) of the output rows."""
+    One row of each sampled tile is the sample: 1/(16 stride) of the output rows.  `only`
+    restricts it to the named projections."""
     import oracle as orc
     out = []
     for p, l in enumerate(wl.block_linears()):
+        if only is not None and l.name not in only:
+            continue
         n, k = l.d_out, l.d_in
         gi = next(i for i, grp in enumerate(BlockWorkload.LAUNCHES) if l.name in grp)
         x = synth.activations(1, k, seed=900 + gi, device=dev)
