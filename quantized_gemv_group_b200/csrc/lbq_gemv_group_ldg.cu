@@ -585,13 +585,13 @@ struct LdgPlan {
 
 // Pair mode: clusters of two CTAs that each get a whole number of tiles, so that no tile
 // is shared outside a cluster and no GPU-scope ticket is left at the end of the launch;
-// chosen for the 16-warp shapes when the grid is full and the largest pair has at most
-// kPairSlack more units than the average.  (On the 8-warp shapes the pair barrier cost
-// more than the tickets it saves.)
+// chosen for the 16-warp shapes of 4 bits or more when the grid is full and the largest
+// pair has at most kPairSlack more units than the average.  (On the 8-warp shapes, and on
+// the 2- and 3-bit ones, whose units are shorter, pairs measured slower than tickets.)
 constexpr bool kLdgPairMode = true;
 constexpr double kPairSlack = 0.06;
 
-static LdgPlan plan_ldg(const int64_t* n, const int64_t* k, int count, int nw) {
+static LdgPlan plan_ldg(const int64_t* n, const int64_t* k, int count, int nw, int bits = 0) {
     LdgPlan pl;
     int64_t max_ksb = 1;
     for (int i = 0; i < count; i++) {
@@ -613,7 +613,7 @@ static LdgPlan plan_ldg(const int64_t* n, const int64_t* k, int count, int nw) {
     // meets at most ceil(ksb W / S) + 1 of them; one more slot of margin
     pl.maxc = (int)(ceil_div(max_ksb * pl.total_warps, std::max<int64_t>(pl.total_units, 1)) + 2);
     const int64_t P = sm_count() / 2;
-    if (kLdgPairMode && nw == 16 && P >= 1 && pl.grid == sm_count() && pl.total_tiles >= P) {
+    if (kLdgPairMode && nw == 16 && bits >= 4 && P >= 1 && pl.grid == sm_count() && pl.total_tiles >= P) {
         auto first_unit = [&](int64_t T) {
             int64_t u = 0;
             for (int i = 0; i < count; i++) {
@@ -710,7 +710,7 @@ lbq_status launch_gemv_group_ldg_multi(const lbq_gemv_problem* probs, int count,
     }
     const int NB = (int)((2 * M + 7) / 8);
     const LdgShape shape = ldg_shape(bits, group, NB);
-    const LdgPlan pl = plan_ldg(n, k, count, shape.NW);
+    const LdgPlan pl = plan_ldg(n, k, count, shape.NW, bits);
     if (pl.total_units == 0) return LBQ_OK;
     if (ws == nullptr || ws_bytes < gemv_group_ldg_ws_bytes_multi(n, k, count, M)) return LBQ_ERR_WORKSPACE;
     if (pl.total_tiles > kMaxTiles || pl.total_units >= ((int64_t)1 << 31)) return LBQ_ERR_UNSUPPORTED;
